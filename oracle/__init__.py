@@ -1,0 +1,44 @@
+"""Float64 CPU oracle for paged KV-cache attention (test infrastructure only).
+
+This package is the independent checker of the CUDA library. Only the test
+suite, the smoke check in ``__graft_entry__`` and the CPU-baseline leg of
+``bench.py`` may import it; the product path never does. It shares no code
+with the CUDA path (no kernels, headers, helpers or tables).
+
+Sources followed (titles of the pages the method is described on):
+
+* "Paged Attention Meets FlexAttention: Unlocking Long-Context Efficiency in
+  Deployed Inference" (abstract): a fused attention kernel that gathers
+  scattered, non-contiguous KV blocks and applies FlexAttention masks.
+* "Ultimate Guide to PagedAttention", sections on KV blocks and the block
+  table: fixed-size blocks (16 tokens typical), a per-request block table that
+  maps logical positions to physical blocks, growth by appending blocks, and
+  prefix sharing with copy-on-write.
+* "FlashAttention: Fast and Memory-Efficient Exact Attention with
+  IO-Awareness" (abstract): attention is computed exactly; tiling only changes
+  the order of memory traffic, never the result.
+
+Because the method is exact, the oracle is the plain definition: resolve each
+block table into a contiguous K/V, then masked softmax attention in float64.
+
+Pins (see ``tests/test_oracle_pins.py``): dense attention from a different
+library routine on a contiguous layout, invariance under permutation of the
+physical blocks, closed forms (identical keys, a dominant key, W >= L), a
+pure-Python brute force on tiny inputs, split-and-merge of the softmax, and
+shared-vs-copied prefixes. No function here is parity-unpinned.
+"""
+
+from .attention64 import (  # noqa: F401
+    MASK_NONE,
+    MASK_CAUSAL,
+    MASK_SLIDING,
+    visible,
+    resolve_block_table,
+    masked_attention,
+    paged_decode,
+    paged_prefill,
+    paged_prefill_rows,
+    paged_decode_rows,
+    kv_append,
+    kv_gather,
+)
