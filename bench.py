@@ -1,0 +1,557 @@
+#!/usr/bin/env python
+"""Benchmark of the paged KV-cache hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+
+* decode: the ragged batch (64 sequences, lengths U[1, 8192], 32/8 heads,
+  head_dim 128, bf16, block 16, 40000-block pool, sliding window 4096 on even
+  sequences): append one token per sequence, then paged decode (main kernel +
+  log-sum-exp combine). Lengths grow by one per step; a sequence takes a new
+  block from the shuffled free list when it crosses a block edge.
+* prefill: 4 sequences with 30720 cached tokens plus a 2048-token chunk,
+  causal: append the chunk through its slot mapping, then paged prefill.
+
+``value`` is decode KV bytes per second (the metric's first part); the
+prefill half is reported in the ``prefill`` object. Inputs are resident in
+HBM when the device-timed region starts; ``e2e`` repeats the steps through
+the public API with pinned host buffers, copies inside the timed region.
+
+``--impl reference`` times the float64 CPU oracle (the only reference this
+method has) on a bounded sample of the same workload.
+"""
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode KV GB/s (frac of HBM peak); paged prefill TFLOP/s (frac of bf16 peak)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.index)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ workloads
+
+def decode_plan(case, steps):
+    """Per-step lengths and append slots for `steps` decode steps; the table
+    gets the blocks the growth will need (entries past a sequence's length
+    are ignored by the kernels)."""
+    bs = case.block_size
+    tab = case.block_tables.numpy().copy()
+    free = case.extra["free_list"]
+    nxt = case.extra["blocks_used"]
+    lens0 = case.seq_lens.numpy().astype(np.int64)
+    nalloc = [(int(L) + bs - 1) // bs for L in lens0]
+    lens = np.zeros((steps, case.batch), dtype=np.int32)
+    slots = np.zeros((steps, case.batch), dtype=np.int64)
+    for s in range(steps):
+        for b in range(case.batch):
+            L = int(lens0[b]) + s
+            p = L - 1
+            j = p // bs
+            if j >= nalloc[b]:
+                tab[b, j] = free[nxt]
+                nxt += 1
+                nalloc[b] = j + 1
+            lens[s, b] = L
+            slots[s, b] = int(tab[b, j]) * bs + p % bs
+    return torch.from_numpy(tab), torch.from_numpy(lens), torch.from_numpy(slots)
+
+
+def visible_tokens(lens, wps):
+    lens = np.asarray(lens, dtype=np.int64)
+    w = np.asarray(wps, dtype=np.int64)
+    return np.where(w > 0, np.minimum(lens, w), lens)
+
+
+class DecodeWork:
+    """The ragged decode batch, resident on the device."""
+
+    def __init__(self, dev, steps, seed):
+        from paged_kv_cache_gather_b200 import inputs as I
+
+        self.case = I.config3(seed=seed, growth_steps=steps + 1)
+        c = self.case
+        tab, lens, slots = decode_plan(c, steps)
+        gen = torch.Generator().manual_seed(seed + 100)
+        B, Hq, Hkv, D = c.batch, c.num_q_heads, c.num_kv_heads, c.head_dim
+        self.q_h = I.randn((steps, B, Hq, D), gen).pin_memory()
+        self.kn_h = I.randn((steps, B, Hkv, D), gen).pin_memory()
+        self.vn_h = I.randn((steps, B, Hkv, D), gen).pin_memory()
+        self.lens_h = lens.pin_memory()
+        self.slots_h = slots.pin_memory()
+        self.tab_h = tab.pin_memory()
+        self.k_cache = c.k_cache.to(dev)
+        self.v_cache = c.v_cache.to(dev)
+        self.tab = tab.to(dev)
+        self.lens = lens.to(dev)
+        self.slots = slots.to(dev)
+        self.q = self.q_h.to(dev)
+        self.kn = self.kn_h.to(dev)
+        self.vn = self.vn_h.to(dev)
+        self.wps = c.window_per_seq.to(dev)
+        self.out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+        self.out_h = torch.empty_like(self.out, device="cpu").pin_memory()
+        self.lse_h = torch.empty_like(self.lse, device="cpu").pin_memory()
+        import paged_kv_cache_gather_b200 as pkv
+
+        self.pkv = pkv
+        self.ws = pkv.decode_workspace(B, Hq, self.k_cache)
+        self.mask = pkv.sliding_window(self.wps)
+        vis = visible_tokens(lens.numpy(), c.window_per_seq.numpy())  # [steps, B]
+        self.kv_bytes = vis.sum(axis=1) * Hkv * D * 2 * 2  # K and V, bf16
+        self.io_bytes = B * Hq * D * 2 * 2 + B * Hq * 4 + ((vis + 15) // 16).sum(1) * Hkv * 4
+        self.append_bytes = B * Hkv * D * 2 * 2 * 2 + B * 8
+        self.h2d = (self.q_h[0].numel() * 2 + self.kn_h[0].numel() * 2 * 2 + B * 4 + B * 8
+                    + self.tab_h.numel() * 4)
+        self.d2h = self.out.numel() * 2 + self.lse.numel() * 4
+
+    def append(self, s):
+        self.pkv.paged_kv_append(self.kn[s], self.vn[s], self.slots[s], self.k_cache, self.v_cache)
+
+    def decode(self, s):
+        self.pkv.paged_attention_decode(self.q[s], self.k_cache, self.v_cache, self.tab,
+                                        self.lens[s], self.case.scale, self.mask, out=self.out,
+                                        lse=self.lse, workspace=self.ws)
+
+    def step_e2e(self, s, dev):
+        q = self.q_h[s].to(dev, non_blocking=True)
+        kn = self.kn_h[s].to(dev, non_blocking=True)
+        vn = self.vn_h[s].to(dev, non_blocking=True)
+        lens = self.lens_h[s].to(dev, non_blocking=True)
+        slots = self.slots_h[s].to(dev, non_blocking=True)
+        tab = self.tab_h.to(dev, non_blocking=True)
+        self.pkv.paged_kv_append(kn, vn, slots, self.k_cache, self.v_cache)
+        self.pkv.paged_attention_decode(q, self.k_cache, self.v_cache, tab, lens,
+                                        self.case.scale, self.mask, out=self.out, lse=self.lse,
+                                        workspace=self.ws)
+        self.out_h.copy_(self.out, non_blocking=True)
+        self.lse_h.copy_(self.lse, non_blocking=True)
+
+
+class PrefillWork:
+    """The long-context chunked prefill batch, resident on the device."""
+
+    def __init__(self, dev, seed):
+        import paged_kv_cache_gather_b200 as pkv
+        from paged_kv_cache_gather_b200 import inputs as I
+
+        self.pkv = pkv
+        self.case = c = I.config5(seed=seed)
+        self.k_cache = c.k_cache.to(dev)
+        self.v_cache = c.v_cache.to(dev)
+        self.tab = c.block_tables.to(dev)
+        self.ctx = c.ctx_lens.to(dev)
+        self.ql = c.q_lens.to(dev)
+        self.q_h = c.q.pin_memory()
+        self.kn_h = c.k_new.pin_memory()
+        self.vn_h = c.v_new.pin_memory()
+        self.slots_h = c.slot_mapping.pin_memory()
+        self.q = self.q_h.to(dev)
+        self.kn = self.kn_h.to(dev)
+        self.vn = self.vn_h.to(dev)
+        self.slots = self.slots_h.to(dev)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(self.q.shape[0], self.q.shape[1], dtype=torch.float32, device=dev)
+        self.out_h = torch.empty_like(self.out, device="cpu").pin_memory()
+        self.lse_h = torch.empty_like(self.lse, device="cpu").pin_memory()
+        self.mask = pkv.causal()
+        C = c.ctx_lens.numpy().astype(np.int64)
+        Q = c.q_lens.numpy().astype(np.int64)
+        pairs = (Q * C + Q * (Q + 1) // 2).sum()  # causally visible (query, key) pairs
+        self.flops = float(4 * c.head_dim * pairs * c.num_q_heads)
+        self.h2d = (self.q.numel() + self.kn.numel() + self.vn.numel()) * 2 + self.slots.numel() * 8
+        self.d2h = self.out.numel() * 2 + self.lse.numel() * 4
+
+    def append(self):
+        self.pkv.paged_kv_append(self.kn, self.vn, self.slots, self.k_cache, self.v_cache)
+
+    def prefill(self):
+        self.pkv.paged_attention_prefill(self.q, self.kn, self.vn, self.k_cache, self.v_cache,
+                                         self.tab, self.ctx, self.ql, self.mask,
+                                         out=self.out, lse=self.lse)
+
+    def step_e2e(self, dev):
+        q = self.q_h.to(dev, non_blocking=True)
+        kn = self.kn_h.to(dev, non_blocking=True)
+        vn = self.vn_h.to(dev, non_blocking=True)
+        slots = self.slots_h.to(dev, non_blocking=True)
+        self.pkv.paged_kv_append(kn, vn, slots, self.k_cache, self.v_cache)
+        self.pkv.paged_attention_prefill(q, kn, vn, self.k_cache, self.v_cache, self.tab,
+                                         self.ctx, self.ql, self.mask, out=self.out, lse=self.lse)
+        self.out_h.copy_(self.out, non_blocking=True)
+        self.lse_h.copy_(self.lse, non_blocking=True)
+
+
+# ------------------------------------------------------------------ CPU baseline
+
+def oracle_decode_sample(budget_s=12.0, seed=None):
+    """Times the float64 oracle on whole decode steps of the ragged batch
+    (all 64 sequences, 32 heads) until `budget_s` has passed."""
+    import oracle
+    from paged_kv_cache_gather_b200 import inputs as I
+
+    c = I.config3(seed=seed)
+    vis = visible_tokens(c.seq_lens.numpy(), c.window_per_seq.numpy())
+    kv_bytes = float(vis.sum() * c.num_kv_heads * c.head_dim * 2 * 2)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.paged_decode(c.q, c.k_cache, c.v_cache, c.block_tables, c.seq_lens, c.scale,
+                            c.mask_kind, c.window, c.window_per_seq)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": kv_bytes * n / el / 1e9, "unit": "GB/s", "cores": cpu_threads(),
+            "kind": "oracle",
+            "sample": f"{n} full decode step(s) of the ragged batch (64 seqs, 32 heads), "
+                      f"{el:.1f} s wall, float64 NumPy"}
+
+
+def oracle_prefill_sample(budget_s=10.0):
+    """Times the oracle on (sequence, head) slices of the prefill batch, scaled."""
+    import oracle
+    from paged_kv_cache_gather_b200 import inputs as I
+
+    c = I.config5(batch=1)
+    C, Q = int(c.ctx_lens[0]), int(c.q_lens[0])
+    rows_per_slice = 64
+    n, t0 = 0, time.perf_counter()
+    while True:
+        h = n % c.num_q_heads
+        oracle.paged_prefill_rows(c.q, c.k_new, c.v_new, c.k_cache, c.v_cache, c.block_tables,
+                                  c.ctx_lens, c.q_lens, c.scale, c.mask_kind,
+                                  rows=[(0, h, i) for i in range(Q - rows_per_slice, Q)])
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    pairs = sum(C + i + 1 for i in range(Q - rows_per_slice, Q))
+    flops = 4.0 * c.head_dim * pairs * n
+    return {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
+            "kind": "oracle",
+            "sample": f"{n} slices of {rows_per_slice} query rows x ~32.7k keys (one head each) "
+                      f"of the prefill batch, {el:.1f} s wall, float64 NumPy"}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        blas = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        blas = 1
+    return int(max(blas, 1))
+
+
+# ------------------------------------------------------------------ main
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x, ws, dev):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return
+    pk, _ = peaks()
+    samples = []
+    for _ in range(args.warmup):
+        oracle_decode_sample(budget_s=0.0)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        samples.append(oracle_decode_sample(budget_s=0.0))
+    el = time.perf_counter() - t0
+    val = statistics.mean(s["value"] for s in samples)
+    line = {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el * 1e3 / max(args.steps, 1), 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "ragged batched decode: 64 seqs, lengths U[1,8192], 32/8 heads, "
+                                   "d128, bf16 pools, block 16, window 4096 on even seqs"},
+            "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": cpu_threads(),
+                             "kind": "oracle",
+                             "sample": "one full decode step of the ragged batch per step"},
+            "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="all", choices=["all", "decode", "prefill"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    ws, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, ws, rank)
+        barrier(ws)
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pk, pk_kind = peaks()
+    total_steps = args.warmup + args.steps
+    seed = 1237 + rank
+    want_decode = args.workload in ("all", "decode")
+    want_prefill = args.workload in ("all", "prefill")
+    dw = DecodeWork(dev, total_steps, seed) if want_decode else None
+    pw = None
+    prefill_reason = None
+    if want_prefill:
+        pw = PrefillWork(dev, 1239 + rank)
+        try:
+            pw.append()
+            pw.prefill()
+            torch.cuda.synchronize()
+        except Exception as e:  # the prefill kernel may not be built for this config
+            prefill_reason = str(e).splitlines()[0]
+            pw = None
+    stream = torch.cuda.current_stream()
+
+    # ---------------- device-timed region
+    for s in range(args.warmup):
+        if dw:
+            dw.append(s)
+            dw.decode(s)
+        if pw:
+            pw.append()
+            pw.prefill()
+    torch.cuda.synchronize()
+    n = args.steps
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    d0, d1, d2 = [ev() for _ in range(n)], [ev() for _ in range(n)], [ev() for _ in range(n)]
+    p0, p1, p2 = [ev() for _ in range(n)], [ev() for _ in range(n)], [ev() for _ in range(n)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(ws)
+    torch.cuda.synchronize()
+    t_start, t_end = ev(), ev()
+    t_start.record(stream)
+    for i in range(n):
+        s = args.warmup + i
+        if dw:
+            d0[i].record(stream)
+            dw.append(s)
+            d1[i].record(stream)
+            dw.decode(s)
+            d2[i].record(stream)
+        if pw:
+            p0[i].record(stream)
+            pw.append()
+            p1[i].record(stream)
+            pw.prefill()
+            p2[i].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), ws, dev)
+
+    # ---------------- end-to-end region (host buffers, copies inside)
+    e2e_steps = n
+    torch.cuda.synchronize()
+    barrier(ws)
+    e_start, e_end, e_mid = ev(), ev(), [ev() for _ in range(e2e_steps)]
+    e_pre = [ev() for _ in range(e2e_steps)]
+    e_start.record(stream)
+    for i in range(e2e_steps):
+        s = args.warmup + i
+        e_pre[i].record(stream)
+        if dw:
+            dw.step_e2e(s, dev)
+        e_mid[i].record(stream)
+        if pw:
+            pw.step_e2e(dev)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop()
+
+    line = {"metric": METRIC, "n_gpus": ws, "steps": n, "warmup": args.warmup,
+            "ms_per_step": round(ms_total / n, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic"}
+    launches = 0
+    if dw:
+        dec_ms = [d1[i].elapsed_time(d2[i]) for i in range(n)]
+        app_ms = [d0[i].elapsed_time(d1[i]) for i in range(n)]
+        steps_idx = range(args.warmup, args.warmup + n)
+        kv = float(sum(dw.kv_bytes[s] for s in steps_idx))
+        io = float(sum(dw.io_bytes[s] for s in steps_idx))
+        dec_total_ms = max_over_ranks(sum(dec_ms) + sum(app_ms), ws, dev)
+        dec_only_ms = max_over_ranks(sum(dec_ms), ws, dev)
+        # whole-job KV throughput of the decode steps (append + decode), all ranks
+        value = kv * ws / (dec_total_ms * 1e-3) / 1e9
+        achieved = (kv + io) / n / (dec_only_ms / n * 1e-3) / 1e9
+        e2e_ms = sum(e_pre[i].elapsed_time(e_mid[i]) for i in range(e2e_steps))
+        e2e_ms = max_over_ranks(e2e_ms, ws, dev)
+        line.update({
+            "value": round(value, 2), "unit": "GB/s",
+            "decode": {"ms_per_step": round(dec_total_ms / n, 4),
+                       "decode_ms": round(dec_only_ms / n, 4),
+                       "append_ms": round(sum(app_ms) / n, 4),
+                       "kv_bytes_per_step": int(kv / n),
+                       "tokens_visible_per_step": int(kv / n / (8 * 128 * 4))},
+            "roofline": {"kernel": "paged_attention_decode (main + combine)", "bound": "hbm",
+                         "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(achieved / pk["hbm_gbs"], 4),
+                         "peak_kind": pk_kind, "traffic": None,
+                         "bytes_per_launch": int((kv + io) / n)},
+            "e2e": {"value": round(kv * ws / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": int(dw.h2d), "d2h_bytes_per_step": int(dw.d2h)},
+        })
+        launches += 3 * n
+    if pw:
+        pre_ms = [p1[i].elapsed_time(p2[i]) for i in range(n)]
+        papp_ms = [p0[i].elapsed_time(p1[i]) for i in range(n)]
+        pre_ms_t = max_over_ranks(sum(pre_ms), ws, dev)
+        pstep_ms = max_over_ranks(sum(pre_ms) + sum(papp_ms), ws, dev)
+        tf = pw.flops * n / (pre_ms_t * 1e-3) / 1e12
+        pe2e = sum(e_mid[i].elapsed_time(e_pre[i + 1] if i + 1 < e2e_steps else e_end)
+                   for i in range(e2e_steps))
+        pe2e = max_over_ranks(pe2e, ws, dev)
+        peak_tf = pk["bf16_tflops"]
+        line["prefill"] = {
+            "value": round(pw.flops * n * ws / (pstep_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(pstep_ms / n, 4), "prefill_ms": round(pre_ms_t / n, 4),
+            "flops_per_step": pw.flops,
+            "roofline": {"kernel": "paged_attention_prefill", "bound": "tensor",
+                         "achieved": round(tf, 1), "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": round(tf / peak_tf, 4),
+                         "frac_of_sustained": round(tf / pk.get("bf16_tflops_sustained", peak_tf), 4),
+                         "peak_kind": pk_kind, "traffic": None},
+            "e2e": {"value": round(pw.flops * n * ws / (pe2e * 1e-3) / 1e12, 2),
+                    "unit": "TFLOP/s", "h2d_bytes_per_step": int(pw.h2d),
+                    "d2h_bytes_per_step": int(pw.d2h)}}
+        launches += 2 * n  # append + prefill (prefill launch count added below)
+    elif want_prefill:
+        line["prefill"] = {"value": None, "unavailable": prefill_reason}
+    if not dw and pw:
+        line.update({"value": line["prefill"]["value"], "unit": "TFLOP/s",
+                     "roofline": line["prefill"]["roofline"], "e2e": line["prefill"]["e2e"]})
+    line["gpu_launches"] = launches
+    line["config"] = {
+        "workload": ("ragged batched decode (64 seqs, lengths U[1,8192] growing 1/step, 32/8 heads, "
+                     "d128, bf16, block 16, 40000-block shuffled pool, window 4096 on even seqs)"
+                     + (" + chunked prefill (4 x (30720 ctx + 2048 chunk), causal)" if pw else "")),
+        "l2": "inputs larger than L2: 0.94 GB of KV per decode step, 537 MB per prefill step "
+              "(126 MB L2), no flush",
+        "parallelism": f"replicas x{ws} (independent batches, no collective)"}
+    line["clocks"] = clk
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_decode_sample()
+        if pw:
+            line["prefill"]["cpu_baseline"] = oracle_prefill_sample()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,206 @@
+/*
+ * pagedkv.h — C ABI of a B200 (sm_100a) paged KV-cache attention library.
+ *
+ * What it computes. Attention over a key/value cache that is cut into
+ * fixed-size blocks of `block_size` tokens (a power of two, 16 by default)
+ * scattered over a physical pool, each sequence reaching its blocks through a
+ * per-sequence block table ("Ultimate Guide to PagedAttention", sections on
+ * KV blocks and on the block table, which maps a sequence's logical positions
+ * to physical memory). The attention kernels gather the scattered blocks
+ * themselves and apply FlexAttention-style mask modifiers inside the fused
+ * kernel ("Paged Attention Meets FlexAttention: Unlocking Long-Context
+ * Efficiency in Deployed Inference", abstract). The result is exact softmax
+ * attention ("FlashAttention: Fast and Memory-Efficient Exact Attention with
+ * IO-Awareness", abstract): tiling changes memory traffic, not the result.
+ *
+ * Layouts (all row-major, all device pointers unless stated):
+ *   k_cache, v_cache  [num_blocks, num_kv_heads, block_size, head_dim]
+ *   block_tables      int32 [batch, max_blocks_per_seq]; entry j of row b is
+ *                     the physical block holding positions j*bs .. j*bs+bs-1
+ *                     of sequence b. Entries past ceil(len/bs) are ignored.
+ *   slot              block * block_size + row; a token at position p of
+ *                     sequence b has slot table[b][p/bs]*bs + p%bs.
+ *   Query head h reads KV head h / (num_q_heads / num_kv_heads).
+ *   lse               float32, natural-log log-sum-exp of the scaled, masked
+ *                     scores, one per (query token, query head).
+ *
+ * Ownership. The caller owns every buffer; the library allocates and frees
+ * nothing. Every call is asynchronous and ordered on `stream` (a
+ * cudaStream_t; NULL means the legacy default stream); none synchronises.
+ *
+ * Errors. Calls return PKV_OK or a negative status. Arguments are checked on
+ * the host before any launch; a rejected call launches nothing.
+ * pkv_last_error() gives a message for the last failure on the calling thread.
+ * Index errors that can only be seen on the device (a block id outside
+ * [0, num_blocks), a slot outside the pool, a length beyond the table) never
+ * trap: the kernel skips the access and ORs a PKV_DBG_* bit into *dbg_err when
+ * dbg_err is not NULL. Read it after the stream completes.
+ */
+#ifndef PAGEDKV_H_
+#define PAGEDKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PKV_VERSION 1
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+/* Status codes. */
+#define PKV_OK 0
+#define PKV_ERR_INVALID_ARG -1         /* null pointer, bad size, misaligned, ... */
+#define PKV_ERR_UNSUPPORTED -2         /* dtype / head_dim / block_size not built */
+#define PKV_ERR_CUDA -3                /* a CUDA runtime call or launch failed */
+#define PKV_ERR_WORKSPACE_TOO_SMALL -4 /* workspace_bytes below the required size */
+#define PKV_ERR_BAD_INDEX -5           /* for wrappers that read dbg_err */
+
+/* Bits ORed into *dbg_err by the kernels. */
+#define PKV_DBG_BLOCK_ID 1    /* block table entry outside [0, num_blocks) */
+#define PKV_DBG_SLOT 2        /* slot_mapping entry outside the pool */
+#define PKV_DBG_LENGTH 4      /* a length needs more table entries than given */
+#define PKV_DBG_TIMEOUT 8     /* a bounded wait on a copy gave up */
+#define PKV_DBG_QLEN_SUM 16   /* prefill: sum of q_lens differs from total_q */
+
+typedef enum { PKV_F32 = 0, PKV_BF16 = 1 } pkv_dtype;
+
+typedef enum {
+  PKV_MASK_NONE = 0,    /* every key of the sequence is visible */
+  PKV_MASK_CAUSAL = 1,  /* key position <= query position */
+  PKV_MASK_SLIDING = 2  /* causal and query - key < window (window keys incl. self) */
+} pkv_mask_kind;
+
+/* FlexAttention-style mask modifier, as data (a C ABI cannot take a callable).
+ * window <= 0 with PKV_MASK_SLIDING means causal only. window_per_seq, when
+ * not NULL, is a device int32 [batch] array that overrides `window` per
+ * sequence (same <= 0 rule). */
+typedef struct {
+  int32_t kind;
+  int32_t window;
+  const int32_t* window_per_seq;
+} pkv_mask_mod;
+
+/* Shape of one K (or V) pool. */
+typedef struct {
+  int32_t num_blocks;
+  int32_t block_size;   /* power of two */
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t dtype;        /* pkv_dtype */
+} pkv_cache_desc;
+
+/*
+ * paged_kv_append — write new tokens' K and V into their slots.
+ * Source: "Ultimate Guide to PagedAttention", dynamic growth: a growing
+ * request takes new blocks and updates its table; no existing data moves.
+ *   k, v          [num_tokens, num_kv_heads, head_dim], cache dtype
+ *   slot_mapping  int64 [num_tokens]; slot < 0 skips the token (padding);
+ *                 slots must be distinct (otherwise which write lands is
+ *                 unspecified). A slot >= num_blocks*block_size is skipped
+ *                 and flagged PKV_DBG_SLOT.
+ * Every other row of the pools is left bit-identical. The copy is exact.
+ * Supported: dtype F32 or BF16, head_dim*elem_size a multiple of 16 bytes,
+ * all pointers 16-byte aligned.
+ */
+PKV_API int paged_kv_append(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+                    void* k_cache, void* v_cache, pkv_cache_desc cache, int32_t* dbg_err,
+                    void* stream);
+
+/*
+ * paged_kv_gather — resolve block tables into contiguous K and V.
+ * Source: "Ultimate Guide to PagedAttention", block table section (logical
+ * positions to physical blocks). Used to check indexing bit for bit.
+ *   k_out, v_out  [batch, num_kv_heads, out_max_len, head_dim], cache dtype;
+ *                 position p < seq_lens[b] holds the stored row exactly,
+ *                 positions >= seq_lens[b] are written as zeros. Lengths
+ *                 beyond out_max_len are cut at out_max_len.
+ */
+PKV_API int paged_kv_gather(const void* k_cache, const void* v_cache, pkv_cache_desc cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* seq_lens, int32_t batch, int32_t out_max_len, void* k_out,
+                    void* v_out, int32_t* dbg_err, void* stream);
+
+/*
+ * paged_attention_decode_workspace_size — bytes of scratch the decode call
+ * needs on the current device (depends on the device's SM count, the group
+ * size num_q_heads/num_kv_heads, head_dim and batch). 0 for float32 pools.
+ */
+PKV_API size_t paged_attention_decode_workspace_size(int32_t batch, int32_t num_q_heads,
+                                             pkv_cache_desc cache);
+
+/*
+ * paged_attention_decode — one query token per sequence over its paged
+ * context. Source: "Paged Attention Meets FlexAttention" (fused kernel that
+ * gathers scattered KV blocks, FlexAttention masks) with the exact softmax
+ * of "FlashAttention" (online softmax, tiling). Long contexts are split
+ * across workers and merged by log-sum-exp; each KV block is read once per
+ * KV head for the whole query-head group.
+ *   q          [batch, num_q_heads, head_dim], cache dtype
+ *   seq_lens   int32 [batch]: keys 0 .. seq_lens[b]-1 (including the token
+ *              just appended); the query sits at position seq_lens[b]-1.
+ *   scale      multiplies q.k (e.g. 1/sqrt(head_dim)).
+ *   out        [batch, num_q_heads, head_dim], cache dtype (bf16 outputs are
+ *              rounded to nearest even from float32).
+ *   lse        float32 [batch, num_q_heads] (may be NULL).
+ *   workspace  device scratch of at least
+ *              paged_attention_decode_workspace_size(...) bytes, 16-byte
+ *              aligned; may be NULL when that size is 0. Contents need no
+ *              initialisation. Calls that share a workspace must not overlap.
+ * A sequence of length 0 gets out = 0 and lse = -inf.
+ * Supported: BF16 with head_dim 64 or 128, block_size >= 8, group size
+ * num_q_heads/num_kv_heads in 1..8; F32 with head_dim <= 256 (any group).
+ */
+PKV_API int paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
+                           pkv_cache_desc cache, const int32_t* block_tables,
+                           int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t batch,
+                           int32_t num_q_heads, float scale, pkv_mask_mod mask, void* out,
+                           float* lse, void* workspace, size_t workspace_bytes,
+                           int32_t* dbg_err, void* stream);
+
+/*
+ * paged_attention_prefill — a chunk of new query tokens per sequence over the
+ * sequence's paged context followed by the chunk itself.
+ * Source: "Paged Attention Meets FlexAttention" (paged, masked attention in
+ * one fused kernel), exact softmax as in "FlashAttention".
+ *   q            [total_q, num_q_heads, head_dim] BF16, packed by sequence
+ *                in batch order (sequence b owns q_lens[b] rows)
+ *   k_new, v_new [total_q, num_kv_heads, head_dim] BF16, packed the same way
+ *   ctx_lens     int32 [batch]: tokens already in the paged cache, read
+ *                through block_tables (positions 0 .. ctx-1)
+ *   q_lens       int32 [batch]: new tokens; new token i of sequence b is at
+ *                position ctx_lens[b] + i, and its K/V come from k_new/v_new.
+ *   scale        multiplies q.k; <= 0 selects 1/sqrt(head_dim).
+ *   out          [total_q, num_q_heads, head_dim] BF16; lse float32
+ *                [total_q, num_q_heads] (may be NULL).
+ * The call does not write the cache: append the chunk with paged_kv_append
+ * (before or after) so later steps see it; the result equals attention over
+ * the appended cache. Supported: BF16, head_dim 128, block_size >= 8.
+ */
+PKV_API int paged_attention_prefill(const void* q, const void* k_new, const void* v_new,
+                            const void* k_cache, const void* v_cache, pkv_cache_desc cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* ctx_lens, const int32_t* q_lens, int32_t batch,
+                            int32_t total_q, int32_t num_q_heads, float scale, pkv_mask_mod mask,
+                            void* out, float* lse, int32_t* dbg_err, void* stream);
+
+/* Name of a status code (static string). */
+PKV_API const char* pkv_status_string(int status);
+
+/* Message of the last failed call on this thread ("" if none). */
+PKV_API const char* pkv_last_error(void);
+
+/* Library version (PKV_VERSION). */
+PKV_API int pkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H_ */

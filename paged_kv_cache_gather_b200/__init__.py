@@ -1,1 +1,28 @@
-"""B200-native paged KV-cache attention (placeholder during bring-up)."""
+"""B200-native paged KV-cache attention.
+
+Calls (thin bindings over the C ABI in ``include/pagedkv.h``):
+
+* ``paged_kv_append``         slot-mapped write of new tokens' K/V
+* ``paged_kv_gather``         block tables resolved to contiguous K/V
+* ``paged_attention_decode``  one query per sequence over paged KV
+* ``paged_attention_prefill`` a chunk of queries over paged context + chunk
+
+Host helpers: ``BlockManager`` (free list, tables, refcounts, copy-on-write)
+and the seeded workload generators in ``inputs``.
+"""
+
+from .blockmgr import BlockManager, OutOfBlocks  # noqa: F401
+from .ops import (  # noqa: F401
+    MaskMod,
+    causal,
+    decode_workspace,
+    decode_workspace_size,
+    no_mask,
+    paged_attention_decode,
+    paged_attention_prefill,
+    paged_kv_append,
+    paged_kv_gather,
+    read_dbg,
+    sliding_window,
+)
+from ._lib import PagedKVError  # noqa: F401

@@ -1,0 +1,220 @@
+// C ABI entry points: argument checks on the host, then one or two kernel
+// launches on the caller's stream. Nothing here allocates device memory or
+// synchronises.
+#include <cudaTypedefs.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "pkv_internal.h"
+
+namespace pkv {
+
+static thread_local char g_last_error[512] = "";
+
+int fail(int status, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return status;
+}
+
+int device_sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+int check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(PKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return PKV_OK;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_pool_tensor_map(void* map_out, const void* base, int64_t rows, int32_t head_dim,
+                          int32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(reinterpret_cast<CUtensorMap*>(map_out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+static int check_cache(const pkv_cache_desc& c, const char* fn) {
+  if (c.num_blocks <= 0 || c.num_kv_heads <= 0 || c.head_dim <= 0 || c.block_size <= 0)
+    return fail(PKV_ERR_INVALID_ARG, "%s: cache sizes must be positive", fn);
+  if (c.block_size & (c.block_size - 1))
+    return fail(PKV_ERR_INVALID_ARG, "%s: block_size %d is not a power of two", fn,
+                c.block_size);
+  if (c.dtype != PKV_F32 && c.dtype != PKV_BF16)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: dtype %d not supported", fn, c.dtype);
+  if ((c.head_dim * dtype_size(c.dtype)) % 16 != 0)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: head_dim*elem_size must be a multiple of 16 bytes",
+                fn);
+  const int64_t rows = (int64_t)c.num_blocks * c.num_kv_heads * c.block_size;
+  if (rows >= (int64_t(1) << 31))
+    return fail(PKV_ERR_UNSUPPORTED, "%s: pool of %lld rows exceeds 2^31", fn, (long long)rows);
+  return PKV_OK;
+}
+
+static int check_mask(const pkv_mask_mod& m, const char* fn) {
+  if (m.kind != PKV_MASK_NONE && m.kind != PKV_MASK_CAUSAL && m.kind != PKV_MASK_SLIDING)
+    return fail(PKV_ERR_INVALID_ARG, "%s: unknown mask kind %d", fn, m.kind);
+  return PKV_OK;
+}
+
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+int pkv_version(void) { return PKV_VERSION; }
+
+const char* pkv_last_error(void) { return g_last_error; }
+
+const char* pkv_status_string(int status) {
+  switch (status) {
+    case PKV_OK: return "PKV_OK";
+    case PKV_ERR_INVALID_ARG: return "PKV_ERR_INVALID_ARG";
+    case PKV_ERR_UNSUPPORTED: return "PKV_ERR_UNSUPPORTED";
+    case PKV_ERR_CUDA: return "PKV_ERR_CUDA";
+    case PKV_ERR_WORKSPACE_TOO_SMALL: return "PKV_ERR_WORKSPACE_TOO_SMALL";
+    case PKV_ERR_BAD_INDEX: return "PKV_ERR_BAD_INDEX";
+    default: return "PKV_ERR_UNKNOWN";
+  }
+}
+
+int paged_kv_append(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+                    void* k_cache, void* v_cache, pkv_cache_desc cache, int32_t* dbg_err,
+                    void* stream) {
+  g_last_error[0] = 0;
+  if (int st = check_cache(cache, "paged_kv_append")) return st;
+  if (num_tokens < 0) return fail(PKV_ERR_INVALID_ARG, "paged_kv_append: num_tokens < 0");
+  if (num_tokens == 0) return PKV_OK;
+  if (!k || !v || !slot_mapping || !k_cache || !v_cache)
+    return fail(PKV_ERR_INVALID_ARG, "paged_kv_append: null pointer");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PKV_ERR_INVALID_ARG, "paged_kv_append: tensors must be 16-byte aligned");
+  return launch_append(k, v, slot_mapping, num_tokens, k_cache, v_cache, cache, dbg_err,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int paged_kv_gather(const void* k_cache, const void* v_cache, pkv_cache_desc cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* seq_lens, int32_t batch, int32_t out_max_len, void* k_out,
+                    void* v_out, int32_t* dbg_err, void* stream) {
+  g_last_error[0] = 0;
+  if (int st = check_cache(cache, "paged_kv_gather")) return st;
+  if (batch < 0 || out_max_len < 0 || max_blocks_per_seq <= 0)
+    return fail(PKV_ERR_INVALID_ARG, "paged_kv_gather: bad batch/out_max_len/max_blocks");
+  if (batch == 0 || out_max_len == 0) return PKV_OK;
+  if (!k_cache || !v_cache || !block_tables || !seq_lens || !k_out || !v_out)
+    return fail(PKV_ERR_INVALID_ARG, "paged_kv_gather: null pointer");
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_out) || !aligned16(v_out))
+    return fail(PKV_ERR_INVALID_ARG, "paged_kv_gather: tensors must be 16-byte aligned");
+  return launch_gather(k_cache, v_cache, cache, block_tables, max_blocks_per_seq, seq_lens, batch,
+                       out_max_len, k_out, v_out, dbg_err, static_cast<cudaStream_t>(stream));
+}
+
+size_t paged_attention_decode_workspace_size(int32_t batch, int32_t num_q_heads,
+                                             pkv_cache_desc cache) {
+  if (check_cache(cache, "paged_attention_decode_workspace_size") != PKV_OK) return 0;
+  if (num_q_heads <= 0 || num_q_heads % cache.num_kv_heads) return 0;
+  return decode_workspace_size(batch, num_q_heads, cache);
+}
+
+int paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
+                           pkv_cache_desc cache, const int32_t* block_tables,
+                           int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t batch,
+                           int32_t num_q_heads, float scale, pkv_mask_mod mask, void* out,
+                           float* lse, void* workspace, size_t workspace_bytes,
+                           int32_t* dbg_err, void* stream) {
+  g_last_error[0] = 0;
+  const char* fn = "paged_attention_decode";
+  if (int st = check_cache(cache, fn)) return st;
+  if (int st = check_mask(mask, fn)) return st;
+  if (batch < 0 || max_blocks_per_seq <= 0)
+    return fail(PKV_ERR_INVALID_ARG, "%s: bad batch or max_blocks_per_seq", fn);
+  if (num_q_heads <= 0 || num_q_heads % cache.num_kv_heads)
+    return fail(PKV_ERR_INVALID_ARG, "%s: num_q_heads %d not a multiple of num_kv_heads %d", fn,
+                num_q_heads, cache.num_kv_heads);
+  if (!(scale == scale)) return fail(PKV_ERR_INVALID_ARG, "%s: scale is NaN", fn);
+  if (batch == 0) return PKV_OK;
+  if (!q || !k_cache || !v_cache || !block_tables || !seq_lens || !out)
+    return fail(PKV_ERR_INVALID_ARG, "%s: null pointer", fn);
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      !aligned16(workspace))
+    return fail(PKV_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", fn);
+  const size_t need = decode_workspace_size(batch, num_q_heads, cache);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+    return fail(PKV_ERR_WORKSPACE_TOO_SMALL, "%s: workspace needs %zu bytes, got %zu", fn, need,
+                workspace_bytes);
+  DecodeArgs a{q,         k_cache, v_cache,    cache, block_tables, max_blocks_per_seq,
+               seq_lens,  batch,   num_q_heads, scale, mask,         out,
+               lse,       workspace, workspace_bytes, dbg_err, static_cast<cudaStream_t>(stream)};
+  return launch_decode(a);
+}
+
+int paged_attention_prefill(const void* q, const void* k_new, const void* v_new,
+                            const void* k_cache, const void* v_cache, pkv_cache_desc cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* ctx_lens, const int32_t* q_lens, int32_t batch,
+                            int32_t total_q, int32_t num_q_heads, float scale, pkv_mask_mod mask,
+                            void* out, float* lse, int32_t* dbg_err, void* stream) {
+  g_last_error[0] = 0;
+  const char* fn = "paged_attention_prefill";
+  if (int st = check_cache(cache, fn)) return st;
+  if (int st = check_mask(mask, fn)) return st;
+  if (batch < 0 || total_q < 0 || max_blocks_per_seq <= 0)
+    return fail(PKV_ERR_INVALID_ARG, "%s: bad batch, total_q or max_blocks_per_seq", fn);
+  if (num_q_heads <= 0 || num_q_heads % cache.num_kv_heads)
+    return fail(PKV_ERR_INVALID_ARG, "%s: num_q_heads %d not a multiple of num_kv_heads %d", fn,
+                num_q_heads, cache.num_kv_heads);
+  if (!(scale == scale)) return fail(PKV_ERR_INVALID_ARG, "%s: scale is NaN", fn);
+  if (batch == 0 || total_q == 0) return PKV_OK;
+  if (!q || !k_new || !v_new || !k_cache || !v_cache || !block_tables || !ctx_lens || !q_lens ||
+      !out)
+    return fail(PKV_ERR_INVALID_ARG, "%s: null pointer", fn);
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || !aligned16(out))
+    return fail(PKV_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", fn);
+  PrefillArgs a{q,        k_new,  v_new, k_cache, v_cache, cache, block_tables, max_blocks_per_seq,
+                ctx_lens, q_lens, batch, total_q, num_q_heads, scale, mask, out,
+                lse,      dbg_err, static_cast<cudaStream_t>(stream)};
+  return launch_prefill(a);
+}
+
+}  // extern "C"

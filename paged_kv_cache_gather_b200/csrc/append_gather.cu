@@ -1,0 +1,124 @@
+// Slot-mapped KV append and block-table gather.
+//
+// Both are exact byte copies, HBM-bound: every thread moves one 16-byte
+// vector of K and one of V (128-bit loads and stores, consecutive threads on
+// consecutive vectors of a head row), grid-stride over a grid sized to a
+// multiple of the SM count.
+//
+// Append follows "Ultimate Guide to PagedAttention", dynamic growth: the new
+// token goes to slot = block * block_size + row and nothing else moves.
+// Gather follows the block-table section of the same page: position p of
+// sequence b lives in block table[b][p / bs], row p % bs.
+#include "pkv_common.cuh"
+#include "pkv_internal.h"
+
+namespace pkv {
+
+__global__ void __launch_bounds__(256) kv_append_kernel(
+    const int4* __restrict__ k, const int4* __restrict__ v, const int64_t* __restrict__ slots,
+    int64_t num_vec, int32_t vec_per_row, int32_t num_kv_heads, int32_t block_shift,
+    int64_t pool_slots, int4* __restrict__ k_cache, int4* __restrict__ v_cache, int32_t* dbg) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t vec_per_tok = (int64_t)vec_per_row * num_kv_heads;
+  const int32_t bs_mask = (1 << block_shift) - 1;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < num_vec; i += stride) {
+    const int64_t t = i / vec_per_tok;
+    const int64_t rem = i - t * vec_per_tok;
+    const int64_t h = rem / vec_per_row;
+    const int64_t c = rem - h * vec_per_row;
+    const int64_t slot = __ldg(slots + t);
+    if (slot < 0) continue;
+    if (slot >= pool_slots) {
+      flag_error(dbg, PKV_DBG_SLOT);
+      continue;
+    }
+    const int64_t blk = slot >> block_shift;
+    const int64_t row = slot & bs_mask;
+    const int64_t dst = (((blk * num_kv_heads + h) << block_shift) + row) * vec_per_row + c;
+    const int4 kv = __ldg(k + i);
+    const int4 vv = __ldg(v + i);
+    k_cache[dst] = kv;
+    v_cache[dst] = vv;
+  }
+}
+
+__global__ void __launch_bounds__(256) kv_gather_kernel(
+    const int4* __restrict__ k_cache, const int4* __restrict__ v_cache,
+    const int32_t* __restrict__ tables, int32_t max_blocks, const int32_t* __restrict__ lens,
+    int64_t num_vec, int32_t vec_per_row, int32_t num_kv_heads, int32_t block_shift,
+    int32_t num_blocks, int32_t out_max_len, int4* __restrict__ k_out, int4* __restrict__ v_out,
+    int32_t* dbg) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int32_t bs_mask = (1 << block_shift) - 1;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < num_vec; i += stride) {
+    // output index i = ((b * Hkv + h) * out_max_len + p) * vec_per_row + c
+    int64_t r = i / vec_per_row;
+    const int64_t c = i - r * vec_per_row;
+    const int64_t p = r % out_max_len;
+    r /= out_max_len;
+    const int64_t h = r % num_kv_heads;
+    const int64_t b = r / num_kv_heads;
+    int4 kv = make_int4(0, 0, 0, 0), vv = kv;
+    const int32_t L = __ldg(lens + b);
+    if (p < L) {
+      const int64_t j = p >> block_shift;
+      if (j >= max_blocks) {
+        flag_error(dbg, PKV_DBG_LENGTH);
+      } else {
+        const int32_t blk = __ldg(tables + b * max_blocks + j);
+        if (blk < 0 || blk >= num_blocks) {
+          flag_error(dbg, PKV_DBG_BLOCK_ID);
+        } else {
+          const int64_t src =
+              ((((int64_t)blk * num_kv_heads + h) << block_shift) + (p & bs_mask)) * vec_per_row +
+              c;
+          kv = __ldg(k_cache + src);
+          vv = __ldg(v_cache + src);
+        }
+      }
+    }
+    k_out[i] = kv;
+    v_out[i] = vv;
+  }
+}
+
+static int grid_for(int64_t work, int threads) {
+  const int sms = device_sm_count();
+  int64_t blocks = (work + threads - 1) / threads;
+  const int64_t cap = (int64_t)sms * 8;  // 8 resident 256-thread CTAs per SM
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return (int)blocks;
+}
+
+int launch_append(const void* k, const void* v, const int64_t* slots, int32_t num_tokens,
+                  void* k_cache, void* v_cache, const pkv_cache_desc& c, int32_t* dbg,
+                  cudaStream_t s) {
+  const int es = dtype_size(c.dtype);
+  const int32_t vec_per_row = c.head_dim * es / 16;
+  const int64_t num_vec = (int64_t)num_tokens * c.num_kv_heads * vec_per_row;
+  if (num_vec == 0) return PKV_OK;
+  const int threads = 256;
+  kv_append_kernel<<<grid_for(num_vec, threads), threads, 0, s>>>(
+      static_cast<const int4*>(k), static_cast<const int4*>(v), slots, num_vec, vec_per_row,
+      c.num_kv_heads, log2_int(c.block_size), (int64_t)c.num_blocks * c.block_size,
+      static_cast<int4*>(k_cache), static_cast<int4*>(v_cache), dbg);
+  return check_launch("paged_kv_append");
+}
+
+int launch_gather(const void* k_cache, const void* v_cache, const pkv_cache_desc& c,
+                  const int32_t* tables, int32_t max_blocks, const int32_t* lens, int32_t batch,
+                  int32_t out_max_len, void* k_out, void* v_out, int32_t* dbg, cudaStream_t s) {
+  const int es = dtype_size(c.dtype);
+  const int32_t vec_per_row = c.head_dim * es / 16;
+  const int64_t num_vec = (int64_t)batch * c.num_kv_heads * out_max_len * vec_per_row;
+  if (num_vec == 0) return PKV_OK;
+  const int threads = 256;
+  kv_gather_kernel<<<grid_for(num_vec, threads), threads, 0, s>>>(
+      static_cast<const int4*>(k_cache), static_cast<const int4*>(v_cache), tables, max_blocks,
+      lens, num_vec, vec_per_row, c.num_kv_heads, log2_int(c.block_size), c.num_blocks,
+      out_max_len, static_cast<int4*>(k_out), static_cast<int4*>(v_out), dbg);
+  return check_launch("paged_kv_gather");
+}
+
+}  // namespace pkv

@@ -1,0 +1,88 @@
+// Host-side internals shared by the translation units of libpagedkv.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pagedkv.h"
+
+namespace pkv {
+
+// Records a message for pkv_last_error() and returns `status`.
+int fail(int status, const char* fmt, ...);
+
+// SM count of the current device (cached per device).
+int device_sm_count();
+
+// Returns PKV_OK, or PKV_ERR_CUDA after recording cudaGetLastError().
+int check_launch(const char* what);
+
+inline int dtype_size(int32_t dt) { return dt == PKV_BF16 ? 2 : 4; }
+
+inline int log2_int(int32_t x) {
+  int r = 0;
+  while ((1 << r) < x) ++r;
+  return r;
+}
+
+int launch_append(const void* k, const void* v, const int64_t* slots, int32_t num_tokens,
+                  void* k_cache, void* v_cache, const pkv_cache_desc& c, int32_t* dbg,
+                  cudaStream_t s);
+
+int launch_gather(const void* k_cache, const void* v_cache, const pkv_cache_desc& c,
+                  const int32_t* tables, int32_t max_blocks, const int32_t* lens, int32_t batch,
+                  int32_t out_max_len, void* k_out, void* v_out, int32_t* dbg, cudaStream_t s);
+
+struct DecodeArgs {
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  pkv_cache_desc cache;
+  const int32_t* tables;
+  int32_t max_blocks;
+  const int32_t* seq_lens;
+  int32_t batch;
+  int32_t num_q_heads;
+  float scale;
+  pkv_mask_mod mask;
+  void* out;
+  float* lse;
+  void* workspace;
+  size_t workspace_bytes;
+  int32_t* dbg;
+  cudaStream_t stream;
+};
+
+size_t decode_workspace_size(int32_t batch, int32_t num_q_heads, const pkv_cache_desc& c);
+int launch_decode(const DecodeArgs& a);
+
+struct PrefillArgs {
+  const void* q;
+  const void* k_new;
+  const void* v_new;
+  const void* k_cache;
+  const void* v_cache;
+  pkv_cache_desc cache;
+  const int32_t* tables;
+  int32_t max_blocks;
+  const int32_t* ctx_lens;
+  const int32_t* q_lens;
+  int32_t batch;
+  int32_t total_q;
+  int32_t num_q_heads;
+  float scale;
+  pkv_mask_mod mask;
+  void* out;
+  float* lse;
+  int32_t* dbg;
+  cudaStream_t stream;
+};
+
+int launch_prefill(const PrefillArgs& a);
+
+// Encodes a 2-D bf16 tensor map over a pool viewed as [rows, head_dim] with a
+// [box_rows, 64]-element box and 128-byte swizzle. Returns false on failure.
+bool make_pool_tensor_map(void* map_out, const void* base, int64_t rows, int32_t head_dim,
+                          int32_t box_rows);
+
+}  // namespace pkv

@@ -139,6 +139,8 @@ def make_decode_case(name, *, lens, num_q_heads, num_kv_heads, head_dim, block_s
     case = PagedCase(name, dtype, num_blocks, block_size, num_kv_heads, num_q_heads, head_dim,
                      k_cache, v_cache, tables, seq_lens, scale, mask_kind, window,
                      window_per_seq, q, k_new, v_new, decode_slots(tables, seq_lens, block_size))
+    case.extra["free_list"] = free
+    case.extra["blocks_used"] = pos
     if peaky:
         make_peaky(case, seed + 7)
     return case
@@ -163,6 +165,8 @@ def make_peaky(case, seed):
         elif case.mask_kind == MASK_SLIDING:
             w = case.window
         lo = max(0, L - w) if (case.mask_kind == MASK_SLIDING and w > 0) else 0
+        if lo >= L - 1:
+            continue
         for kvh in range(case.num_kv_heads):
             p = int(rng.integers(lo, L - 1))  # not the appended token
             qh = case.q[b, kvh * g].float()

@@ -1,0 +1,209 @@
+"""Python binding of the paged KV-cache calls: argument marshalling only.
+
+Each function checks devices, dtypes and shapes, allocates outputs with torch
+when the caller passes none, and calls the C ABI of ``libpagedkv.so`` on the
+current CUDA stream. Every step of the computation runs in the library's
+CUDA kernels; nothing here computes attention.
+"""
+
+import ctypes
+import math
+from dataclasses import dataclass
+from typing import Optional, Union
+
+import torch
+
+from . import _lib as L
+
+_DTYPES = {torch.float32: L.PKV_F32, torch.bfloat16: L.PKV_BF16}
+
+
+@dataclass
+class MaskMod:
+    """FlexAttention-style mask modifier as data.
+
+    kind: ``MaskMod.NONE``, ``CAUSAL`` or ``SLIDING``. ``window`` (sliding only)
+    keeps keys with ``q_pos - k_pos < window``; ``<= 0`` means causal only.
+    ``window_per_seq`` (int32 CUDA tensor [batch]) overrides ``window``.
+    """
+
+    kind: int = L.PKV_MASK_NONE
+    window: int = 0
+    window_per_seq: Optional[torch.Tensor] = None
+
+    NONE = L.PKV_MASK_NONE
+    CAUSAL = L.PKV_MASK_CAUSAL
+    SLIDING = L.PKV_MASK_SLIDING
+
+    def to_c(self, batch, device):
+        wps = None
+        if self.window_per_seq is not None:
+            w = self.window_per_seq
+            _check(w.dtype == torch.int32 and w.device == device and w.is_contiguous()
+                   and w.numel() >= batch, "window_per_seq must be int32 [batch] on the device")
+            wps = w.data_ptr()
+        return L.MaskModC(int(self.kind), int(self.window), wps)
+
+
+def no_mask() -> MaskMod:
+    return MaskMod(L.PKV_MASK_NONE)
+
+
+def causal() -> MaskMod:
+    return MaskMod(L.PKV_MASK_CAUSAL)
+
+
+def sliding_window(window: Union[int, torch.Tensor]) -> MaskMod:
+    if isinstance(window, torch.Tensor):
+        return MaskMod(L.PKV_MASK_SLIDING, 0, window)
+    return MaskMod(L.PKV_MASK_SLIDING, int(window))
+
+
+def _check(cond, msg):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def cache_desc(k_cache: torch.Tensor) -> L.CacheDescC:
+    _check(k_cache.dim() == 4, "cache must be [num_blocks, num_kv_heads, block_size, head_dim]")
+    _check(k_cache.dtype in _DTYPES, f"cache dtype {k_cache.dtype} not supported")
+    nb, hkv, bs, d = k_cache.shape
+    return L.CacheDescC(nb, bs, hkv, d, _DTYPES[k_cache.dtype])
+
+
+def _check_pool(k_cache, v_cache):
+    _check(k_cache.is_cuda and v_cache.device == k_cache.device, "caches must be on one GPU")
+    _check(k_cache.shape == v_cache.shape and k_cache.dtype == v_cache.dtype,
+           "k_cache and v_cache must match")
+    _check(k_cache.is_contiguous() and v_cache.is_contiguous(), "caches must be contiguous")
+
+
+def _i32(t, name, device):
+    _check(t.dtype == torch.int32 and t.device == device and t.is_contiguous(),
+           f"{name} must be a contiguous int32 tensor on {device}")
+    return t
+
+
+def paged_kv_append(k, v, slot_mapping, k_cache, v_cache, dbg_err=None):
+    """Write K/V of new tokens into their slots (exact copy; slot < 0 skips)."""
+    _check_pool(k_cache, v_cache)
+    dev = k_cache.device
+    T = k.shape[0]
+    _check(k.shape == (T, k_cache.shape[1], k_cache.shape[3]) and v.shape == k.shape,
+           "k, v must be [num_tokens, num_kv_heads, head_dim]")
+    _check(k.dtype == k_cache.dtype and v.dtype == k_cache.dtype, "k/v dtype must match cache")
+    _check(k.is_contiguous() and v.is_contiguous() and k.device == dev and v.device == dev,
+           "k, v must be contiguous on the cache's device")
+    _check(slot_mapping.dtype == torch.int64 and slot_mapping.device == dev
+           and slot_mapping.numel() == T and slot_mapping.is_contiguous(),
+           "slot_mapping must be int64 [num_tokens] on the device")
+    L.check(L.lib().paged_kv_append(_ptr(k), _ptr(v), _ptr(slot_mapping), T, _ptr(k_cache),
+                                    _ptr(v_cache), cache_desc(k_cache), _ptr(dbg_err), _stream()))
+
+
+def paged_kv_gather(k_cache, v_cache, block_tables, seq_lens, out_max_len, dbg_err=None):
+    """Contiguous [B, Hkv, out_max_len, d] copies of each sequence's K and V."""
+    _check_pool(k_cache, v_cache)
+    dev = k_cache.device
+    _i32(block_tables, "block_tables", dev)
+    _i32(seq_lens, "seq_lens", dev)
+    B = seq_lens.numel()
+    _check(block_tables.dim() == 2 and block_tables.shape[0] == B, "block_tables must be [B, M]")
+    nb, hkv, bs, d = k_cache.shape
+    ko = torch.empty(B, hkv, out_max_len, d, dtype=k_cache.dtype, device=dev)
+    vo = torch.empty_like(ko)
+    L.check(L.lib().paged_kv_gather(_ptr(k_cache), _ptr(v_cache), cache_desc(k_cache),
+                                    _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), B,
+                                    int(out_max_len), _ptr(ko), _ptr(vo), _ptr(dbg_err),
+                                    _stream()))
+    return ko, vo
+
+
+def decode_workspace_size(batch, num_q_heads, k_cache):
+    return int(L.lib().paged_attention_decode_workspace_size(batch, num_q_heads,
+                                                             cache_desc(k_cache)))
+
+
+def decode_workspace(batch, num_q_heads, k_cache):
+    n = decode_workspace_size(batch, num_q_heads, k_cache)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=k_cache.device)
+
+
+def paged_attention_decode(q, k_cache, v_cache, block_tables, seq_lens, scale=None,
+                           mask_mod: Optional[MaskMod] = None, *, out=None, lse=None,
+                           workspace=None, dbg_err=None):
+    """One query token per sequence over its paged context. Returns (out, lse)."""
+    _check_pool(k_cache, v_cache)
+    dev = k_cache.device
+    _i32(block_tables, "block_tables", dev)
+    _i32(seq_lens, "seq_lens", dev)
+    B, Hq, d = q.shape
+    _check(q.dtype == k_cache.dtype and q.device == dev and q.is_contiguous(),
+           "q must be contiguous, on the cache's device, in the cache dtype")
+    _check(d == k_cache.shape[3], "head_dim mismatch")
+    _check(block_tables.dim() == 2 and block_tables.shape[0] == B and seq_lens.numel() == B,
+           "block_tables [B, M] and seq_lens [B] must match q's batch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    mask_mod = mask_mod or no_mask()
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = decode_workspace(B, Hq, k_cache)
+    L.check(L.lib().paged_attention_decode(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), cache_desc(k_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(seq_lens), B, Hq, float(scale), mask_mod.to_c(B, dev),
+        _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _ptr(dbg_err), _stream()))
+    return out, lse
+
+
+def paged_attention_prefill(q, k_new, v_new, k_cache, v_cache, block_tables, ctx_lens, q_lens,
+                            mask_mod: Optional[MaskMod] = None, scale=None, *, out=None,
+                            lse=None, dbg_err=None):
+    """A chunk of new queries per sequence over its paged context plus the
+    chunk itself. q/k_new/v_new are packed by sequence. Returns (out, lse)."""
+    _check_pool(k_cache, v_cache)
+    dev = k_cache.device
+    _i32(block_tables, "block_tables", dev)
+    _i32(ctx_lens, "ctx_lens", dev)
+    _i32(q_lens, "q_lens", dev)
+    T, Hq, d = q.shape
+    B = ctx_lens.numel()
+    _check(q_lens.numel() == B and block_tables.dim() == 2 and block_tables.shape[0] == B,
+           "ctx_lens, q_lens and block_tables must agree on the batch")
+    for t, name in ((q, "q"), (k_new, "k_new"), (v_new, "v_new")):
+        _check(t.dtype == k_cache.dtype and t.device == dev and t.is_contiguous(),
+               f"{name} must be contiguous, on the cache's device, in the cache dtype")
+    _check(k_new.shape == (T, k_cache.shape[1], d) and v_new.shape == k_new.shape,
+           "k_new/v_new must be [total_q, num_kv_heads, head_dim]")
+    mask_mod = mask_mod or no_mask()
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(T, Hq, dtype=torch.float32, device=dev)
+    L.check(L.lib().paged_attention_prefill(
+        _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), cache_desc(k_cache),
+        _ptr(block_tables), block_tables.shape[1], _ptr(ctx_lens), _ptr(q_lens), B, T, Hq,
+        float(scale) if scale is not None else 0.0, mask_mod.to_c(B, dev), _ptr(out), _ptr(lse),
+        _ptr(dbg_err), _stream()))
+    return out, lse
+
+
+def read_dbg(dbg_err):
+    """Raise PagedKVError if a kernel flagged an index error in ``dbg_err``."""
+    v = int(dbg_err.item())
+    if v:
+        names = [n for n, bit in (("block id", L.PKV_DBG_BLOCK_ID), ("slot", L.PKV_DBG_SLOT),
+                                  ("length", L.PKV_DBG_LENGTH), ("timeout", L.PKV_DBG_TIMEOUT),
+                                  ("q_lens sum", L.PKV_DBG_QLEN_SUM)) if v & bit]
+        raise L.PagedKVError(L.PKV_ERR_BAD_INDEX, "device flagged: " + ", ".join(names))
