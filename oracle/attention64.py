@@ -264,7 +264,8 @@ def kv_append(k, v, slot_mapping, k_cache, v_cache):
 def kv_gather(k_cache, v_cache, block_tables, seq_lens, out_max_len):
     """Contiguous copies ``[B, Hkv, out_max_len, d]`` of each sequence's K and V.
 
-    Positions ``>= seq_lens[b]`` are zero. Copies stored values exactly (any
+    Positions ``>= seq_lens[b]`` are zero; a longer sequence is cut at
+    ``out_max_len``. Copies stored values exactly (any
     dtype, torch or NumPy), so it can be compared bit for bit.
     """
     lens = _i64(seq_lens)
@@ -278,7 +279,7 @@ def kv_gather(k_cache, v_cache, block_tables, seq_lens, out_max_len):
         ko = np.zeros((B, Hkv, out_max_len, d), dtype=k_cache.dtype)
         vo = np.zeros((B, Hkv, out_max_len, d), dtype=v_cache.dtype)
     for b in range(B):
-        L = int(lens[b])
+        L = min(int(lens[b]), out_max_len)
         pos = np.arange(L)
         blocks, rows = tables[b][pos // bs], pos % bs
         if hasattr(k_cache, "detach"):

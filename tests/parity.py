@@ -49,8 +49,9 @@ def assert_attention_close(out, lse, ref_out, ref_lse, dtype, what=""):
     den = np.linalg.norm(ref_out.reshape(-1, ref_out.shape[-1]), axis=1)
     nz = den > 0
     assert np.all(num[~nz] == 0), f"{what}: nonzero output where the reference is zero"
-    rel = num[nz] / den[nz]
-    assert rel.max() <= NORM_RTOL, f"{what}: normwise rel err {rel.max()}"
+    if nz.any():
+        rel = num[nz] / den[nz]
+        assert rel.max() <= NORM_RTOL, f"{what}: normwise rel err {rel.max()}"
 
 
 def run_decode(case, dev, do_append=True, dbg=True):

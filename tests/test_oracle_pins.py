@@ -399,6 +399,8 @@ def test_gather_brute_force():
                                         dtype=torch.bfloat16)
     ko, vo = oracle.kv_gather(kc, vc, tab, lens, 16)
     assert ko.dtype == torch.bfloat16 and ko.shape == (3, 2, 16, 4)
+    cut, _ = oracle.kv_gather(kc, vc, tab, lens, 9)  # the 14-token sequence is cut at 9
+    assert torch.equal(cut, ko[:, :, :9])
     for b in range(3):
         for h in range(2):
             for p in range(16):
