@@ -190,6 +190,32 @@ PKV_API int paged_attention_prefill(const void* q, const void* k_new, const void
                             int32_t total_q, int32_t num_q_heads, float scale, pkv_mask_mod mask,
                             void* out, float* lse, int32_t* dbg_err, void* stream);
 
+/*
+ * paged_attention_decode_noalloc — paged_attention_decode without a
+ * caller-provided workspace. The pages have no counterpart to this call: it
+ * exists for callers that cannot allocate device memory (a runtime whose
+ * device memory all belongs to its own pool, a C or embedded host without a
+ * device allocator, a loop that cannot afford cudaMalloc's synchronisation).
+ * Same arguments, layouts, results and errors as paged_attention_decode,
+ * minus workspace/workspace_bytes. The split-KV scratch is a fixed array of
+ * PKV_NOALLOC_SCRATCH_BYTES inside the library's device image, held on every
+ * GPU that loads the library until the process exits. The first call on a
+ * device looks up that array's address (once per device, with the device
+ * current); make that first call before any stream capture begins. Every
+ * call shares the array: calls that overlap on the GPU race and give wrong
+ * results, so order them on one stream. Nothing in the array needs to start
+ * at zero. A problem that needs more scratch than the array holds returns
+ * PKV_ERR_WORKSPACE_TOO_SMALL and launches nothing. The call allocates and
+ * frees nothing.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES (8u << 20)
+PKV_API int paged_attention_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                           pkv_cache_desc cache, const int32_t* block_tables,
+                                           int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                           int32_t batch, int32_t num_q_heads, float scale,
+                                           pkv_mask_mod mask, void* out, float* lse,
+                                           int32_t* dbg_err, void* stream);
+
 /* Name of a status code (static string). */
 PKV_API const char* pkv_status_string(int status);
 
