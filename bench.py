@@ -140,10 +140,11 @@ def visible_tokens(lens, wps):
 class DecodeWork:
     """The ragged decode batch, resident on the device."""
 
-    def __init__(self, dev, steps, seed):
+    def __init__(self, dev, steps, seed, batch=64, num_blocks=40000):
         from paged_kv_cache_gather_b200 import inputs as I
 
-        self.case = I.config3(seed=seed, growth_steps=steps + 1)
+        self.case = I.config3(batch=batch, num_blocks=num_blocks, seed=seed,
+                              growth_steps=steps + 1)
         c = self.case
         tab, lens, slots = decode_plan(c, steps)
         gen = torch.Generator().manual_seed(seed + 100)
@@ -384,6 +385,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="all", choices=["all", "decode", "prefill"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--small", action="store_true",
+                    help="profiling size: 16 decode sequences in a 12000-block pool "
+                         "(still larger than L2); not a bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     ws, rank, local = dist_setup()
@@ -398,7 +402,10 @@ def main():
     seed = 1237 + rank
     want_decode = args.workload in ("all", "decode")
     want_prefill = args.workload in ("all", "prefill")
-    dw = DecodeWork(dev, total_steps, seed) if want_decode else None
+    if args.small:
+        dw = DecodeWork(dev, total_steps, seed, batch=16, num_blocks=12000) if want_decode else None
+    else:
+        dw = DecodeWork(dev, total_steps, seed) if want_decode else None
     pw = None
     prefill_reason = None
     if want_prefill:
