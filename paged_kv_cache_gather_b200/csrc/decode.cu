@@ -15,7 +15,10 @@
 //    that a second kernel merges by log-sum-exp. The split depends only on
 //    the lengths and the window, never on block ids, so the result is
 //    bit-identical under any placement of the blocks.
-//  * Each warp runs its own NSTAGE-deep TMA ring: a 16-row x 64-column box
+//  * 12 workers per CTA, one CTA per SM: each warp is one serial stream of
+//    dependent MMA/shuffle work, so the SM needs several warps per
+//    sub-partition to issue every cycle (4 warps reached 59% of HBM peak,
+//    12 warps 86%). Each warp runs its own NSTAGE-deep TMA ring: a 16-row x 64-column box
 //    per 128-byte half of the head row, 128-byte swizzled, so the tensor-core
 //    fragment loads (ldmatrix) are bank-conflict free. Block ids are loaded
 //    one tile ahead of the copy that needs them.
@@ -26,6 +29,7 @@
 //    movmatrix, without a trip through shared memory.
 //  * fp32 pools use a plain CUDA-core kernel (one CTA per (b, q head)).
 #include <cmath>
+#include <cstdlib>
 
 #include "pkv_common.cuh"
 #include "pkv_internal.h"
@@ -34,7 +38,8 @@ namespace pkv {
 
 constexpr int kTile = 16;            // tokens per tile
 constexpr int kMinTilesPerWorker = 2;
-constexpr int kWarpsPerCta = 4;      // workers (warps) per CTA, one CTA per SM
+constexpr int kWarpsPerCta = 12;     // default workers (warps) per CTA, one CTA per SM
+constexpr int kMaxWarpsPerCta = 12;  // largest built variant (sizes the workspace)
 
 struct DecodeParams {
   const __nv_bfloat16* q;
@@ -476,64 +481,95 @@ __global__ void __launch_bounds__(WPC * 32, 1)
 }
 
 // Merges the partials of segments split between workers, and writes zeros /
-// -inf for empty sequences. One warp per (b, KV head) segment.
+// -inf for empty sequences. One warp per (segment, query head): lanes load
+// the pieces' LSEs in parallel, reduce max and sum with shuffles, then sum
+// the weighted partial outputs with lanes over head_dim.
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
+  constexpr int V = D / 32;  // floats per lane
   const int lane = threadIdx.x & 31;
-  const int64_t seg = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
-  if (seg >= (int64_t)p.batch * p.num_kv_heads) return;
-  const int b = (int)(seg / p.num_kv_heads);
-  const int kvh = (int)(seg % p.num_kv_heads);
+  const int64_t item = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
   const int H = p.num_kv_heads;
-  const int64_t T = (int64_t)p.ws_prefix[p.batch] * H;
+  if (item >= (int64_t)p.batch * H * p.group) return;
+  const int h = (int)(item % p.group);
+  const int64_t seg = item / p.group;
+  const int b = (int)(seg / H);
+  const int kvh = (int)(seg % H);
   const int n = p.ws_prefix[b + 1] - p.ws_prefix[b];
-  const int64_t obase = ((int64_t)b * p.num_q_heads + kvh * p.group) * D;
-  const int64_t lbase = (int64_t)b * p.num_q_heads + kvh * p.group;
+  const int64_t orow = ((int64_t)b * p.num_q_heads + kvh * p.group + h);
+  __nv_bfloat16* dst = p.out + orow * D + lane * V;
   if (n == 0) {
-    for (int i = lane; i < p.group * D; i += 32) p.out[obase + i] = __float2bfloat16_rn(0.f);
-    if (p.lse && lane < p.group) p.lse[lbase + lane] = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < V; ++i) dst[i] = __float2bfloat16_rn(0.f);
+    if (p.lse && lane == 0) p.lse[orow] = -INFINITY;
     return;
   }
+  const int64_t T = (int64_t)p.ws_prefix[p.batch] * H;
   const int W = workers_for(T, p.workers);
   const int64_t s0 = (int64_t)p.ws_prefix[b] * H + (int64_t)kvh * n;
   const int64_t s1 = s0 + n;
   auto owner = [&](int64_t x) { return (int)(((x + 1) * W - 1) / T); };
   const int wf = owner(s0), wl = owner(s1 - 1);
   if (wf == wl) return;  // written whole by one worker
-  for (int h = 0; h < p.group; ++h) {
-    float mx = -INFINITY;
-    for (int w = wf; w <= wl; ++w) {
-      const int64_t st = (int64_t)w * T / W, en = (int64_t)(w + 1) * T / W;
-      if (st == en) continue;
-      const int kind = (w == wf && st < s0) ? 1 : 0;
-      mx = fmaxf(mx, __ldcg(p.ws_lse + ((int64_t)w * 2 + kind) * p.group + h));
+  // slot of worker w's piece of this segment, or -1 if w has no tiles
+  auto slot_of = [&](int w) -> int64_t {
+    const int64_t st = (int64_t)w * T / W, en = (int64_t)(w + 1) * T / W;
+    if (st == en) return -1;
+    return (int64_t)w * 2 + ((w == wf && st < s0) ? 1 : 0);
+  };
+  // pass 1: log-sum-exp over the pieces, 32 pieces per round
+  float m = -INFINITY, sum = 0.f;
+  for (int base = wf; base <= wl; base += 32) {
+    const int w = base + lane;
+    float x = -INFINITY;
+    if (w <= wl) {
+      const int64_t sl = slot_of(w);
+      if (sl >= 0) x = __ldcg(p.ws_lse + sl * p.group + h);
     }
-    float sum = 0.f;
-    for (int w = wf; w <= wl; ++w) {
-      const int64_t st = (int64_t)w * T / W, en = (int64_t)(w + 1) * T / W;
-      if (st == en) continue;
-      const int kind = (w == wf && st < s0) ? 1 : 0;
-      sum += expf(__ldcg(p.ws_lse + ((int64_t)w * 2 + kind) * p.group + h) - mx);
-    }
-    const float lse = mx + logf(sum);
-    float acc[D / 32];
+    float mx = x;
 #pragma unroll
-    for (int i = 0; i < D / 32; ++i) acc[i] = 0.f;
-    for (int w = wf; w <= wl; ++w) {
-      const int64_t st = (int64_t)w * T / W, en = (int64_t)(w + 1) * T / W;
-      if (st == en) continue;
-      const int kind = (w == wf && st < s0) ? 1 : 0;
-      const int64_t slot = (int64_t)w * 2 + kind;
-      const float wgt = expf(__ldcg(p.ws_lse + slot * p.group + h) - lse);
-      const float* src = p.ws_o + (slot * p.group + h) * D;
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float nm = fmaxf(m, mx);
+    float e = (x == -INFINITY) ? 0.f : __expf(x - nm);
 #pragma unroll
-      for (int i = 0; i < D / 32; ++i) acc[i] += wgt * __ldcg(src + lane + 32 * i);
-    }
-#pragma unroll
-    for (int i = 0; i < D / 32; ++i)
-      p.out[obase + h * D + lane + 32 * i] = __float2bfloat16_rn(acc[i]);
-    if (p.lse && lane == 0) p.lse[lbase + h] = lse;
+    for (int o = 16; o; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+    sum = (m == -INFINITY ? 0.f : sum * __expf(m - nm)) + e;
+    m = nm;
   }
+  const float lse = m + logf(sum);
+  // pass 2: weighted sum of the normalised partial outputs
+  float acc[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) acc[i] = 0.f;
+  for (int base = wf; base <= wl; base += 32) {
+    const int w = base + lane;
+    int64_t sl = -1;
+    float wgt = 0.f;
+    if (w <= wl) {
+      sl = slot_of(w);
+      if (sl >= 0) wgt = __expf(__ldcg(p.ws_lse + sl * p.group + h) - lse);
+    }
+    const int cnt = min(32, wl - base + 1);
+    for (int j = 0; j < cnt; ++j) {
+      const float wj = __shfl_sync(0xffffffffu, wgt, j);
+      const int64_t sj = __shfl_sync(0xffffffffu, sl, j);
+      if (sj < 0) continue;
+      const float* src = p.ws_o + (sj * p.group + h) * D + lane * V;
+      if constexpr (V == 4) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
+        acc[0] += wj * v.x;
+        acc[1] += wj * v.y;
+        acc[2] += wj * v.z;
+        acc[3] += wj * v.w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] += wj * __ldcg(src + i);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < V; ++i) dst[i] = __float2bfloat16_rn(acc[i]);
+  if (p.lse && lane == 0) p.lse[orow] = lse;
 }
 
 // ---------------------------------------------------------------- fp32 path
@@ -684,21 +720,40 @@ int launch_bf16_impl(const DecodeArgs& a) {
 
   decode_bf16_kernel<D, NSTAGE, WPC><<<sms, WPC * 32, smem, a.stream>>>(kmap, vmap, p);
   if (int st = check_launch("paged_attention_decode")) return st;
-  const int64_t segs = (int64_t)a.batch * a.cache.num_kv_heads;
-  decode_combine_kernel<D><<<(unsigned)((segs + 3) / 4), 128, 0, a.stream>>>(p);
+  const int64_t items = (int64_t)a.batch * a.cache.num_kv_heads * g;
+  decode_combine_kernel<D><<<(unsigned)((items + 3) / 4), 128, 0, a.stream>>>(p);
   return check_launch("paged_attention_decode: combine");
+}
+
+// Warps per CTA (one CTA per SM) and ring depth per warp. PKV_DECODE_WARPS
+// picks another built variant (for tuning sweeps); the default is the
+// fastest measured on B200.
+int decode_warps_per_cta() {
+  static int w = [] {
+    const char* e = getenv("PKV_DECODE_WARPS");
+    int v = e ? atoi(e) : kWarpsPerCta;
+    if (v != 4 && v != 6 && v != 8 && v != 12) v = kWarpsPerCta;
+    return v;
+  }();
+  return w;
 }
 
 template <int D>
 int launch_bf16(const DecodeArgs& a) {
-  return launch_bf16_impl<D, (D == 128 ? 6 : 10), kWarpsPerCta>(a);
+  // 192 KB of ring per CTA for head_dim 128 (8 KB stages), 160-192 KB for 64
+  switch (decode_warps_per_cta()) {
+    case 6: return launch_bf16_impl<D, (D == 128 ? 4 : 8), 6>(a);
+    case 8: return launch_bf16_impl<D, (D == 128 ? 3 : 6), 8>(a);
+    case 4: return launch_bf16_impl<D, (D == 128 ? 6 : 10), 4>(a);
+    default: return launch_bf16_impl<D, (D == 128 ? 2 : 4), 12>(a);
+  }
 }
 
 }  // namespace
 
 size_t decode_workspace_size(int32_t batch, int32_t num_q_heads, const pkv_cache_desc& c) {
   if (c.dtype != PKV_BF16) return 0;
-  const int workers = device_sm_count() * kWarpsPerCta;
+  const int workers = device_sm_count() * kMaxWarpsPerCta;
   const int g = num_q_heads / c.num_kv_heads;
   const size_t o_bytes = (size_t)2 * workers * g * c.head_dim * 4;
   const size_t l_bytes = ((size_t)2 * workers * g * 4 + 255) & ~size_t(255);
