@@ -85,4 +85,9 @@ int launch_prefill(const PrefillArgs& a);
 bool make_pool_tensor_map(void* map_out, const void* base, int64_t rows, int32_t head_dim,
                           int32_t box_rows);
 
+// Encodes a bf16 tensor map of rank 1..5 with 128-byte swizzle; dims and
+// box innermost first, strides in bytes for dims 1..rank-1.
+bool make_tensor_map_bf16(void* map_out, const void* base, int rank, const uint64_t* dims,
+                          const uint64_t* strides_bytes, const uint32_t* box);
+
 }  // namespace pkv

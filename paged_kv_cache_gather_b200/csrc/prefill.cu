@@ -1,12 +1,742 @@
-// Paged chunked prefill (placeholder until the tensor-core kernel lands).
+// Paged chunked prefill on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// Method: "Paged Attention Meets FlexAttention" (abstract) — attention of new
+// query tokens over the sequence's scattered KV blocks, gathered by the
+// fused kernel through the block table, with the mask modifier applied in
+// the kernel — computed exactly with the tiled online softmax of
+// "FlashAttention" (abstract). Keys are the cached context (positions
+// 0 .. ctx-1, read through the block table) followed by the new chunk
+// (positions ctx .. ctx+q-1, read from k_new / v_new).
+//
+// B200 design:
+//  * Persistent CTAs, one per SM. A unit of work is (sequence, KV head, pair
+//    of query heads of that KV head's group, 128-row query tile); the two
+//    heads share every K/V tile the CTA loads (GQA). Units are handed out
+//    round-robin, longest (last query tiles) first.
+//  * Warp roles: warps 0-3 and 4-7 are the softmax warpgroups of head 0 and
+//    head 1 (one query row per thread); warp 8 issues TMA loads; warp 9
+//    allocates tensor memory and issues the MMAs.
+//  * Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.
+//    S = Q K^T is written by tcgen05.mma (M=128, N=128 keys, K=16 x 8); the
+//    softmax warps read S, write P as bf16 into the first 64 columns of the
+//    same S region, and O += P V reads P straight from tensor memory
+//    (A operand in TMEM) with V as an MN-major shared-memory operand.
+//  * MMA issue order S0(j), PV1(j-1), S1(j), PV0(j): while one warpgroup
+//    turns its S into P the tensor core runs the other head's work.
+//  * K/V tiles are 128 keys: context tiles are 8 TMA boxes of 16 rows, one
+//    per 16-token piece of a paged block (block id from the table); chunk
+//    tiles are one 3-D box of k_new / v_new. All loads use 128-byte
+//    swizzle. Rows past the context end are loaded as out-of-bounds boxes,
+//    which TMA fills with zeros, so no stale value reaches P*V.
+//  * Online softmax in base 2 with a lazy rescale: O and l are rescaled only
+//    when a row maximum grows by more than 8 (a factor 256), otherwise the
+//    stale maximum is kept (P stays <= 256, exact in fp32/bf16 range). The
+//    final normalisation uses the same maximum, so the result is exact.
+#include <cmath>
+
 #include "pkv_common.cuh"
 #include "pkv_internal.h"
+#include "tc_sm100.cuh"
 
 namespace pkv {
 
+namespace {
+
+constexpr int kD = 128;             // head dim
+constexpr int kM = 128;             // query rows per tile
+constexpr int kN = 128;             // keys per tile
+constexpr int kStages = 2;          // K/V ring depth
+constexpr int kTileBytes = kN * kD * 2;   // 32 KB (K or V or Q tile)
+constexpr int kHalfBytes = kTileBytes / 2;
+constexpr int kThreads = 320;
+constexpr int kMaxBatch = 4096;
+constexpr float kRescaleThreshold = 8.f;  // log2 units
+
+struct PrefillParams {
+  const int32_t* tables;
+  int32_t max_blocks;
+  const int32_t* ctx_lens;
+  const int32_t* q_lens;
+  int32_t batch;
+  int32_t total_q;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t group;
+  int32_t pairs;        // units per KV head: group/2 (two heads) or group (one head)
+  int32_t two_heads;    // 1 when a unit holds two query heads
+  int32_t bs_shift;
+  int32_t box_rows;     // rows of one paged TMA box (min(block_size, 16))
+  int32_t num_blocks;
+  int32_t pool_rows;    // num_blocks * Hkv * block_size (first out-of-bounds row)
+  float scale_log2;
+  int32_t mask_kind;
+  int32_t window;
+  const int32_t* window_per_seq;
+  __nv_bfloat16* out;
+  float* lse;
+  int32_t* dbg;
+};
+
+struct SmemLayout {
+  // offsets from the 1024-aligned base
+  static constexpr int kQ0 = 0;
+  static constexpr int kQ1 = kTileBytes;
+  static constexpr int kKV = 2 * kTileBytes;  // stage s: K at kKV + s*2*tile, V after it
+  static constexpr int kBars = kKV + kStages * 2 * kTileBytes;
+  static constexpr int kNumBars = 2 + 2 * kStages + 9;
+  static constexpr int kTmemSlot = kBars + kNumBars * 8;
+  static constexpr int kQoff = kTmemSlot + 16;  // int32 [batch + 1]
+  static constexpr int kMaxQt = kQoff - 8;      // int32 (placed before the prefix)
+};
+
+// barrier indices
+enum : int {
+  BAR_Q_FULL = 0,
+  BAR_Q_EMPTY = 1,
+  BAR_KV_FULL = 2,                 // + stage
+  BAR_KV_EMPTY = 2 + kStages,      // + stage
+  BAR_S_FULL = 2 + 2 * kStages,    // + head
+  BAR_P_FULL = BAR_S_FULL + 2,     // + head
+  BAR_O_FULL = BAR_P_FULL + 2,     // + head
+  BAR_O_FREE = BAR_O_FULL + 2,     // + head
+  BAR_KV_FIXED = BAR_O_FREE + 2,   // a tile whose rows past the context end were zeroed
+};
+
+struct Unit {
+  bool valid;
+  int b, kvh, hp, qt;
+  int C, Q, qoff;
+  int ctx_lo, n_ctx;   // context tiles [ctx_lo, ctx_lo + n_ctx)
+  int ch_lo, n_ch;     // chunk tiles   [ch_lo, ch_lo + n_ch)
+  int window;          // <= 0: no window
+  __device__ int n() const { return n_ctx + n_ch; }
+};
+
+__device__ __forceinline__ int window_of(const PrefillParams& p, int b) {
+  if (p.mask_kind != PKV_MASK_SLIDING) return 0;
+  return p.window_per_seq ? p.window_per_seq[b] : p.window;
+}
+
+__device__ __forceinline__ Unit unit_of(const PrefillParams& p, const int32_t* qoff, int max_qt,
+                                        int64_t u) {
+  Unit x;
+  const int64_t per_qt = (int64_t)p.batch * p.num_kv_heads * p.pairs;
+  const int qt_rev = (int)(u / per_qt);
+  int64_t rem = u - (int64_t)qt_rev * per_qt;
+  x.b = (int)(rem / ((int64_t)p.num_kv_heads * p.pairs));
+  rem -= (int64_t)x.b * p.num_kv_heads * p.pairs;
+  x.kvh = (int)(rem / p.pairs);
+  x.hp = (int)(rem % p.pairs);
+  x.qt = max_qt - 1 - qt_rev;
+  x.Q = qoff[x.b + 1] - qoff[x.b];
+  x.qoff = qoff[x.b];
+  x.valid = x.qt >= 0 && x.qt * kM < x.Q;
+  if (!x.valid) return x;
+  int C = p.ctx_lens[x.b];
+  if (C < 0) C = 0;
+  const int cap = p.max_blocks << p.bs_shift;
+  if (C > cap) {
+    flag_error(p.dbg, PKV_DBG_LENGTH);
+    C = cap;
+  }
+  x.C = C;
+  x.window = window_of(p, x.b);
+  const int qmin = C + x.qt * kM;             // position of the tile's first row
+  const int ctx_tiles = (C + kN - 1) / kN;
+  const int q_tiles = (x.Q + kN - 1) / kN;
+  int lo_key = 0;                              // lowest key any row of the tile can see
+  if (x.window > 0) lo_key = max(0, qmin - x.window + 1);
+  x.ctx_lo = min(lo_key / kN, ctx_tiles);
+  x.n_ctx = ctx_tiles - x.ctx_lo;
+  const int ch_hi = (p.mask_kind == PKV_MASK_NONE) ? q_tiles - 1 : min(x.qt, q_tiles - 1);
+  x.ch_lo = (lo_key > C) ? (lo_key - C) / kN : 0;
+  x.n_ch = max(0, ch_hi - x.ch_lo + 1);
+  return x;
+}
+
+// Tile j of a unit: is it a context tile, and the position of its first key.
+__device__ __forceinline__ void tile_of(const Unit& x, int j, bool& ctx, int& idx, int& kp0) {
+  if (j < x.n_ctx) {
+    ctx = true;
+    idx = x.ctx_lo + j;
+    kp0 = idx * kN;
+  } else {
+    ctx = false;
+    idx = x.ch_lo + (j - x.n_ctx);
+    kp0 = x.C + idx * kN;
+  }
+}
+
+// A context tile whose 16-row box straddles the context end holds rows past
+// it that come from the pool (stale, possibly non-finite); they are zeroed in
+// shared memory before the MMAs read the tile.
+__device__ __forceinline__ bool needs_fix(const Unit& x, bool ctx, int kp0, int box_rows) {
+  return ctx && kp0 < x.C && kp0 + kN > x.C && (x.C % box_rows) != 0;
+}
+
+// Warp-collective bounded wait: every lane of the warp calls it and gets the
+// same answer, so the warp never splits around the warp-wide tcgen05
+// instructions that follow. On a timeout (or an abort raised by another
+// warp) it records PKV_DBG_TIMEOUT and tells every role to stop.
+__device__ __forceinline__ bool wait_or_flag(uint32_t bar, uint32_t parity, int32_t* dbg,
+                                             int* abort_flag) {
+  bool ok = *reinterpret_cast<volatile int*>(abort_flag) == 0 && mbar_wait(bar, parity);
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok && (threadIdx.x & 31) == 0) {
+    flag_error(dbg, PKV_DBG_TIMEOUT);
+    *reinterpret_cast<volatile int*>(abort_flag) = 1;
+  }
+  return ok;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// 3-D TMA tile load (inner coordinate first).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int32_t c0,
+                                            int32_t c1, int32_t c2, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
+struct Maps {
+  CUtensorMap q;      // 3-D {D, Hq, total_q}, box {64, 1, 128}
+  CUtensorMap knew;   // 3-D {D, Hkv, total_q}, box {64, 1, 128}
+  CUtensorMap vnew;
+  CUtensorMap kpool;  // 2-D {D, pool rows}, box {64, box_rows}
+  CUtensorMap vpool;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ Maps maps, const PrefillParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  using L = SmemLayout;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+  int32_t* qoff = reinterpret_cast<int32_t*>(smem + L::kQoff);
+  int32_t* max_qt_s = reinterpret_cast<int32_t*>(smem + L::kMaxQt);
+  int* abort_flag = reinterpret_cast<int*>(smem + L::kMaxQt + 4);
+
+  // ---- set-up: barriers, tensor memory, per-sequence query offsets
+  if (warp == 8) {
+    if (lane == 0) {
+      mbar_init(bar(BAR_Q_FULL), 1);
+      mbar_init(bar(BAR_Q_EMPTY), 1);
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(bar(BAR_KV_FULL + s), 1);
+        mbar_init(bar(BAR_KV_EMPTY + s), 1);
+      }
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(bar(BAR_S_FULL + h), 1);
+        mbar_init(bar(BAR_P_FULL + h), 128);
+        mbar_init(bar(BAR_O_FULL + h), 1);
+        mbar_init(bar(BAR_O_FREE + h), 128);
+      }
+      mbar_init(bar(BAR_KV_FIXED), 1);
+      *abort_flag = 0;
+      fence_barrier_init();
+      prefetch_tmap(&maps.q);
+      prefetch_tmap(&maps.knew);
+      prefetch_tmap(&maps.vnew);
+      prefetch_tmap(&maps.kpool);
+      prefetch_tmap(&maps.vpool);
+    }
+    // exclusive prefix of q_lens and the largest number of query tiles
+    int run = 0, mq = 0;
+    for (int base = 0; base < p.batch; base += 32) {
+      const int b = base + lane;
+      int q = b < p.batch ? max(0, p.q_lens[b]) : 0;
+      mq = max(mq, (q + kM - 1) / kM);
+      int incl = q;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (b < p.batch) qoff[b] = run + incl - q;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mq = max(mq, __shfl_xor_sync(0xffffffffu, mq, o));
+    if (lane == 0) {
+      qoff[p.batch] = run;
+      *max_qt_s = mq;
+      if (run != p.total_q && blockIdx.x == 0) flag_error(p.dbg, PKV_DBG_QLEN_SUM);
+    }
+  } else if (warp == 9) {
+    tc::tmem_alloc(smem_u32(tmem_slot), 512);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int max_qt = *max_qt_s;
+  const int64_t num_units = (int64_t)max_qt * p.batch * p.num_kv_heads * p.pairs;
+  const uint32_t q_bytes = (p.two_heads ? 2u : 1u) * kTileBytes;
+
+  if (warp == 8) {
+    // ================================================================ TMA producer
+    int unit_k = 0;
+    uint32_t kv_count = 0;
+    for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
+      const Unit x = unit_of(p, qoff, max_qt, u);
+      if (!x.valid) continue;
+      const int h0 = x.kvh * p.group + x.hp * (p.two_heads ? 2 : 1);
+      // query tiles (slot reusable once the previous unit's MMAs are done)
+      if (unit_k > 0 && !wait_or_flag(bar(BAR_Q_EMPTY), (unit_k - 1) & 1, p.dbg, abort_flag)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(BAR_Q_FULL), q_bytes);
+        const int row0 = x.qoff + x.qt * kM;
+        for (int hh = 0; hh < (p.two_heads ? 2 : 1); ++hh)
+          for (int half = 0; half < 2; ++half)
+            tma_load_3d(smem_u32(smem + (hh ? L::kQ1 : L::kQ0) + half * kHalfBytes), &maps.q,
+                        half * 64, h0 + hh, row0, bar(BAR_Q_FULL));
+      }
+      // key/value tiles
+      const int n = x.n();
+      for (int j = 0; j < n; ++j, ++kv_count) {
+        const int s = kv_count % kStages;
+        if (kv_count >= (uint32_t)kStages &&
+            !wait_or_flag(bar(BAR_KV_EMPTY + s), ((kv_count / kStages) - 1) & 1, p.dbg,
+                          abort_flag))
+          break;
+        bool ctx;
+        int idx, kp0;
+        tile_of(x, j, ctx, idx, kp0);
+        const uint32_t kdst = smem_u32(smem + L::kKV + s * 2 * kTileBytes);
+        const uint32_t vdst = kdst + kTileBytes;
+        const uint32_t fb = bar(BAR_KV_FULL + s);
+        if (lane == 0) mbar_arrive_expect_tx(fb, 2 * kTileBytes);
+        __syncwarp();
+        if (!ctx) {
+          if (lane == 0) {
+            const int row0 = x.qoff + idx * kN;
+            for (int half = 0; half < 2; ++half) {
+              tma_load_3d(kdst + half * kHalfBytes, &maps.knew, half * 64, x.kvh, row0, fb);
+              tma_load_3d(vdst + half * kHalfBytes, &maps.vnew, half * 64, x.kvh, row0, fb);
+            }
+          }
+        } else {
+          // one lane per box of `box_rows` paged rows
+          const int nbox = kN / p.box_rows;
+          for (int bi = lane; bi < nbox; bi += 32) {
+            const int pos = kp0 + bi * p.box_rows;
+            const uint32_t off = bi * p.box_rows * 128;
+            if (pos + p.box_rows <= x.C) {
+              const int j_blk = pos >> p.bs_shift;
+              int id = p.tables[(int64_t)x.b * p.max_blocks + j_blk];
+              int row;
+              if (id < 0 || id >= p.num_blocks) {
+                flag_error(p.dbg, PKV_DBG_BLOCK_ID);
+                row = p.pool_rows;  // out of bounds: zero fill
+              } else {
+                row = ((id * p.num_kv_heads + x.kvh) << p.bs_shift) + (pos & ((1 << p.bs_shift) - 1));
+              }
+              for (int half = 0; half < 2; ++half) {
+                tma_load_2d(kdst + half * kHalfBytes + off, &maps.kpool, half * 64, row, fb);
+                tma_load_2d(vdst + half * kHalfBytes + off, &maps.vpool, half * 64, row, fb);
+              }
+            } else if (pos >= x.C) {
+              for (int half = 0; half < 2; ++half) {
+                tma_load_2d(kdst + half * kHalfBytes + off, &maps.kpool, half * 64, p.pool_rows, fb);
+                tma_load_2d(vdst + half * kHalfBytes + off, &maps.vpool, half * 64, p.pool_rows, fb);
+              }
+            } else {
+              // straddles the context end: load the block; rows past the end are
+              // zeroed below once the tile has landed
+              const int j_blk = pos >> p.bs_shift;
+              int id = p.tables[(int64_t)x.b * p.max_blocks + j_blk];
+              int row;
+              if (id < 0 || id >= p.num_blocks) {
+                flag_error(p.dbg, PKV_DBG_BLOCK_ID);
+                row = p.pool_rows;
+              } else {
+                row = ((id * p.num_kv_heads + x.kvh) << p.bs_shift) + (pos & ((1 << p.bs_shift) - 1));
+              }
+              for (int half = 0; half < 2; ++half) {
+                tma_load_2d(kdst + half * kHalfBytes + off, &maps.kpool, half * 64, row, fb);
+                tma_load_2d(vdst + half * kHalfBytes + off, &maps.vpool, half * 64, row, fb);
+              }
+            }
+          }
+          if (needs_fix(x, ctx, kp0, p.box_rows)) {
+            if (!wait_or_flag(fb, (kv_count / kStages) & 1, p.dbg, abort_flag)) break;
+            // zero V rows [C - kp0, end of that box) in both 64-column halves
+            const int r0 = x.C - kp0;
+            const int r1 = (r0 / p.box_rows + 1) * p.box_rows;
+            uint8_t* vbase = smem + L::kKV + s * 2 * kTileBytes + kTileBytes;
+            for (int i = lane; i < (r1 - r0) * 2 * 8; i += 32) {
+              const int rr = r0 + i / 16;
+              const int half = (i / 8) & 1;
+              const int ch = i & 7;
+              *reinterpret_cast<int4*>(vbase + half * kHalfBytes + rr * 128 + ch * 16) =
+                  make_int4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(BAR_KV_FIXED));
+          }
+        }
+      }
+      ++unit_k;
+    }
+  } else if (warp == 9) {
+    // ================================================================ MMA issuer
+    const uint32_t idesc_s = tc::idesc_bf16(kM, kN, false, false);
+    const uint32_t idesc_o = tc::idesc_bf16(kM, kD, false, true);
+    const uint32_t S0 = tmem, S1 = tmem + 128, O0 = tmem + 256, O1 = tmem + 384;
+    const uint32_t q0 = smem_u32(smem + L::kQ0), q1 = smem_u32(smem + L::kQ1);
+    int unit_k = 0;
+    uint32_t kv_count = 0, p_cnt0 = 0, p_cnt1 = 0, fix_count = 0;
+    auto issue_s = [&](uint32_t d, uint32_t qa, uint32_t ka) {
+#pragma unroll
+      for (int kk = 0; kk < kD / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+        tc::mma_ss(d, tc::smem_desc(qa + off, 16, 1024, tc::kSwizzle128B),
+                   tc::smem_desc(ka + off, 16, 1024, tc::kSwizzle128B), idesc_s, kk > 0);
+      }
+    };
+    auto issue_pv = [&](uint32_t d, uint32_t p_tmem, uint32_t va, bool acc) {
+#pragma unroll
+      for (int kk = 0; kk < kN / 16; ++kk)
+        tc::mma_ts(d, p_tmem + kk * 8,
+                   tc::smem_desc(va + kk * 2048, kHalfBytes, 1024, tc::kSwizzle128B), idesc_o,
+                   acc || kk > 0);
+    };
+    for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
+      const Unit x = unit_of(p, qoff, max_qt, u);
+      if (!x.valid) continue;
+      const int n = x.n();
+      if (!wait_or_flag(bar(BAR_Q_FULL), unit_k & 1, p.dbg, abort_flag)) break;
+      tc::fence_after_sync();
+      uint32_t prev_v = 0;
+      int prev_s = 0;
+      bool ok = true;
+      for (int j = 0; j < n && ok; ++j, ++kv_count) {
+        const int s = kv_count % kStages;
+        if (!wait_or_flag(bar(BAR_KV_FULL + s), (kv_count / kStages) & 1, p.dbg, abort_flag)) {
+          ok = false;
+          break;
+        }
+        {
+          bool ctx_t;
+          int idx_t, kp0_t;
+          tile_of(x, j, ctx_t, idx_t, kp0_t);
+          if (needs_fix(x, ctx_t, kp0_t, p.box_rows)) {
+            if (!wait_or_flag(bar(BAR_KV_FIXED), fix_count & 1, p.dbg, abort_flag)) {
+              ok = false;
+              break;
+            }
+            ++fix_count;
+          }
+        }
+        tc::fence_after_sync();
+        const uint32_t ka = smem_u32(smem + L::kKV + s * 2 * kTileBytes);
+        const uint32_t va = ka + kTileBytes;
+        if (lane == 0) {
+          issue_s(S0, q0, ka);
+          tc::commit(bar(BAR_S_FULL + 0));
+        }
+        __syncwarp();
+        if (p.two_heads) {
+          if (j > 0) {
+            if (!wait_or_flag(bar(BAR_P_FULL + 1), p_cnt1 & 1, p.dbg, abort_flag)) { ok = false; break; }
+            ++p_cnt1;
+            tc::fence_after_sync();
+            if (j - 1 == 0 && unit_k > 0 &&
+                !wait_or_flag(bar(BAR_O_FREE + 1), (unit_k - 1) & 1, p.dbg, abort_flag)) { ok = false; break; }
+            if (lane == 0) {
+              issue_pv(O1, S1, prev_v, j - 1 > 0);
+              tc::commit(bar(BAR_KV_EMPTY + prev_s));
+            }
+            __syncwarp();
+          }
+          if (lane == 0) {
+            issue_s(S1, q1, ka);
+            tc::commit(bar(BAR_S_FULL + 1));
+          }
+          __syncwarp();
+        }
+        if (!wait_or_flag(bar(BAR_P_FULL + 0), p_cnt0 & 1, p.dbg, abort_flag)) { ok = false; break; }
+        ++p_cnt0;
+        tc::fence_after_sync();
+        if (j == 0 && unit_k > 0 &&
+            !wait_or_flag(bar(BAR_O_FREE + 0), (unit_k - 1) & 1, p.dbg, abort_flag)) { ok = false; break; }
+        if (lane == 0) {
+          issue_pv(O0, S0, va, j > 0);
+          if (!p.two_heads) tc::commit(bar(BAR_KV_EMPTY + s));
+        }
+        __syncwarp();
+        prev_v = va;
+        prev_s = s;
+      }
+      if (!ok) break;
+      if (p.two_heads) {
+        if (!wait_or_flag(bar(BAR_P_FULL + 1), p_cnt1 & 1, p.dbg, abort_flag)) break;
+        ++p_cnt1;
+        tc::fence_after_sync();
+        if (n == 1 && unit_k > 0 &&
+            !wait_or_flag(bar(BAR_O_FREE + 1), (unit_k - 1) & 1, p.dbg, abort_flag)) break;
+        if (lane == 0) {
+          issue_pv(O1, S1, prev_v, n - 1 > 0);
+          tc::commit(bar(BAR_KV_EMPTY + prev_s));
+        }
+        __syncwarp();
+      }
+      if (lane == 0) {
+        tc::commit(bar(BAR_O_FULL + 0));
+        tc::commit(bar(BAR_O_FULL + 1));
+        tc::commit(bar(BAR_Q_EMPTY));
+      }
+      __syncwarp();
+      ++unit_k;
+    }
+  } else {
+    // ================================================================ softmax warpgroups
+    const int hsel = warp >> 2;              // which head of the pair
+    const int row = (warp & 3) * 32 + lane;  // query row of the tile = TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t S = tmem + hsel * 128 + lane_base;
+    const uint32_t O = tmem + 256 + hsel * 128 + lane_base;
+    int unit_k = 0;
+    uint32_t s_cnt = 0;
+    for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
+      const Unit x = unit_of(p, qoff, max_qt, u);
+      if (!x.valid) continue;
+      if (hsel == 1 && !p.two_heads) {
+        ++unit_k;
+        continue;
+      }
+      const int n = x.n();
+      const int i_row = x.qt * kM + row;      // query index within the chunk
+      const int qpos = x.C + i_row;
+      const int qmin = x.C + x.qt * kM, qmax = qmin + kM - 1;
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < n; ++j, ++s_cnt) {
+        if (!wait_or_flag(bar(BAR_S_FULL + hsel), s_cnt & 1, p.dbg, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
+        bool ctx;
+        int idx, kp0;
+        tile_of(x, j, ctx, idx, kp0);
+        const int key_end = ctx ? x.C : x.C + x.Q;
+        bool full = kp0 + kN <= key_end;
+        if (p.mask_kind != PKV_MASK_NONE) full = full && (kp0 + kN - 1 <= qmin);
+        if (x.window > 0) full = full && (qmax - kp0 < x.window);
+        // pass 1: row maximum over the visible keys of the tile
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tc::ld32(S + c * 32, r);
+          tc::wait_ld();
+          if (full) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(r[i]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int kpos = kp0 + c * 32 + i;
+              bool vis = kpos < key_end;
+              if (p.mask_kind != PKV_MASK_NONE) vis = vis && kpos <= qpos;
+              if (x.window > 0) vis = vis && (qpos - kpos < x.window);
+              if (vis) mx = fmaxf(mx, __uint_as_float(r[i]));
+            }
+          }
+        }
+        const float mxs = mx * p.scale_log2;  // scale > 0 keeps the order
+        // lazy rescale: move the reference maximum only when it grows by > 2^8
+        float alpha = 1.f;
+        if (mxs > m + kRescaleThreshold || (m == -INFINITY && mxs != -INFINITY)) {
+          if (m != -INFINITY) alpha = fast_exp2(m - mxs);
+          m = mxs;
+        }
+        const float mb = (m == -INFINITY) ? 0.f : m;
+        float ls0 = 0.f, ls1 = 0.f;
+        // pass 2: P = exp2(s*c - m) (0 for masked keys), bf16 into the S columns
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t r0[32], r1[32], pk[32];
+          tc::ld32(S + hf * 64, r0);
+          tc::ld32(S + hf * 64 + 32, r1);
+          tc::wait_ld();
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const float s0 = __uint_as_float(cc ? r1[i] : r0[i]);
+              const float s1 = __uint_as_float(cc ? r1[i + 1] : r0[i + 1]);
+              float e0 = fast_exp2(fmaf(s0, p.scale_log2, -mb));
+              float e1 = fast_exp2(fmaf(s1, p.scale_log2, -mb));
+              if (!full) {
+                const int kpos = kp0 + hf * 64 + cc * 32 + i;
+                bool v0 = kpos < key_end, v1 = kpos + 1 < key_end;
+                if (p.mask_kind != PKV_MASK_NONE) {
+                  v0 = v0 && kpos <= qpos;
+                  v1 = v1 && kpos + 1 <= qpos;
+                }
+                if (x.window > 0) {
+                  v0 = v0 && (qpos - kpos < x.window);
+                  v1 = v1 && (qpos - kpos - 1 < x.window);
+                }
+                e0 = v0 ? e0 : 0.f;
+                e1 = v1 ? e1 : 0.f;
+              }
+              ls0 += e0;
+              ls1 += e1;
+              pk[cc * 16 + i / 2] = pack_bf16x2(e0, e1);
+            }
+          }
+          tc::st32(S + hf * 32, pk);
+        }
+        l = l * alpha + ls0 + ls1;
+        // tcgen05.ld/st are warp-collective: the whole warp takes this branch
+        // when any of its rows moved its maximum (the others scale by 1)
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+          // rescale this row of O; the previous P*V has completed (it was issued
+          // before this S) and the next one waits for this thread's arrival
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tc::ld32(O + c * 32, o);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tc::st32(O + c * 32, o);
+          }
+        }
+        tc::wait_st();
+        tc::fence_before_sync();
+        mbar_arrive(bar(BAR_P_FULL + hsel));
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16, lse
+      if (!wait_or_flag(bar(BAR_O_FULL + hsel), unit_k & 1, p.dbg, abort_flag)) break;
+      tc::fence_after_sync();
+      const int h = x.kvh * p.group + x.hp * (p.two_heads ? 2 : 1) + hsel;
+      const bool valid_row = i_row < x.Q && x.qoff + i_row < p.total_q;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* dst = p.out + ((int64_t)(x.qoff + i_row) * p.num_q_heads + h) * kD;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tc::ld32(O + c * 32, o);
+        tc::wait_ld();
+        if (valid_row) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+            *reinterpret_cast<uint4*>(dst + c * 32 + i) = v;
+          }
+        }
+      }
+      if (valid_row && p.lse)
+        p.lse[(int64_t)(x.qoff + i_row) * p.num_q_heads + h] =
+            l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+      tc::fence_before_sync();
+      mbar_arrive(bar(BAR_O_FREE + hsel));
+      ++unit_k;
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 9) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+              const uint64_t* strides_bytes, const uint32_t* box) {
+  return make_tensor_map_bf16(m, base, rank, dims, strides_bytes, box);
+}
+
+}  // namespace
+
 int launch_prefill(const PrefillArgs& a) {
-  (void)a;
-  return fail(PKV_ERR_UNSUPPORTED, "paged_attention_prefill: not built yet");
+  const char* fn = "paged_attention_prefill";
+  if (a.cache.dtype != PKV_BF16)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: only bf16 pools are supported", fn);
+  if (a.cache.head_dim != kD)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: head_dim %d (128 supported)", fn, a.cache.head_dim);
+  if (a.cache.block_size < 8)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: block_size must be >= 8", fn);
+  if (a.batch > kMaxBatch)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: batch %d > %d", fn, a.batch, kMaxBatch);
+  const int Hkv = a.cache.num_kv_heads;
+  const int g = a.num_q_heads / Hkv;
+  PrefillParams p;
+  p.tables = a.tables;
+  p.max_blocks = a.max_blocks;
+  p.ctx_lens = a.ctx_lens;
+  p.q_lens = a.q_lens;
+  p.batch = a.batch;
+  p.total_q = a.total_q;
+  p.num_q_heads = a.num_q_heads;
+  p.num_kv_heads = Hkv;
+  p.group = g;
+  p.two_heads = (g % 2 == 0) ? 1 : 0;
+  p.pairs = p.two_heads ? g / 2 : g;
+  p.bs_shift = log2_int(a.cache.block_size);
+  p.box_rows = a.cache.block_size < 16 ? a.cache.block_size : 16;
+  p.num_blocks = a.cache.num_blocks;
+  const int64_t pool_rows = (int64_t)a.cache.num_blocks * Hkv * a.cache.block_size;
+  p.pool_rows = (int32_t)pool_rows;
+  const float scale = a.scale > 0.f ? a.scale : 1.f / sqrtf((float)kD);
+  p.scale_log2 = scale * kLog2e;
+  p.mask_kind = a.mask.kind;
+  p.window = a.mask.window;
+  p.window_per_seq = a.mask.window_per_seq;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
+  p.dbg = a.dbg;
+
+  alignas(64) Maps maps;
+  {
+    const uint64_t dq[3] = {(uint64_t)kD, (uint64_t)a.num_q_heads, (uint64_t)a.total_q};
+    const uint64_t sq[2] = {(uint64_t)kD * 2, (uint64_t)a.num_q_heads * kD * 2};
+    const uint64_t dk[3] = {(uint64_t)kD, (uint64_t)Hkv, (uint64_t)a.total_q};
+    const uint64_t sk[2] = {(uint64_t)kD * 2, (uint64_t)Hkv * kD * 2};
+    const uint32_t box3[3] = {64, 1, (uint32_t)kM};
+    const uint64_t dp[2] = {(uint64_t)kD, (uint64_t)pool_rows};
+    const uint64_t sp[1] = {(uint64_t)kD * 2};
+    const uint32_t boxp[2] = {64, (uint32_t)p.box_rows};
+    if (!make_map(&maps.q, a.q, 3, dq, sq, box3) || !make_map(&maps.knew, a.k_new, 3, dk, sk, box3) ||
+        !make_map(&maps.vnew, a.v_new, 3, dk, sk, box3) ||
+        !make_map(&maps.kpool, a.k_cache, 2, dp, sp, boxp) ||
+        !make_map(&maps.vpool, a.v_cache, 2, dp, sp, boxp))
+      return fail(PKV_ERR_CUDA, "%s: tensor map encoding failed", fn);
+  }
+  const size_t smem = SmemLayout::kQoff + (size_t)(a.batch + 1) * 4 + 1024;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    const size_t max_smem = SmemLayout::kQoff + (size_t)(kMaxBatch + 1) * 4 + 1024;
+    if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)max_smem) != cudaSuccess)
+      return check_launch("paged_attention_prefill: smem attribute");
+    attr_set[dev] = true;
+  }
+  const int grid = device_sm_count();
+  prefill_kernel<<<grid, kThreads, smem, a.stream>>>(maps, p);
+  return check_launch(fn);
 }
 
 }  // namespace pkv
