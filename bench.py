@@ -207,12 +207,12 @@ class DecodeWork:
 class PrefillWork:
     """The long-context chunked prefill batch, resident on the device."""
 
-    def __init__(self, dev, seed):
+    def __init__(self, dev, seed, batch=4):
         import paged_kv_cache_gather_b200 as pkv
         from paged_kv_cache_gather_b200 import inputs as I
 
         self.pkv = pkv
-        self.case = c = I.config5(seed=seed)
+        self.case = c = I.config5(batch=batch, seed=seed)
         self.k_cache = c.k_cache.to(dev)
         self.v_cache = c.v_cache.to(dev)
         self.tab = c.block_tables.to(dev)
@@ -386,8 +386,8 @@ def main():
     ap.add_argument("--workload", default="all", choices=["all", "decode", "prefill"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--small", action="store_true",
-                    help="profiling size: 16 decode sequences in a 12000-block pool "
-                         "(still larger than L2); not a bench line")
+                    help="profiling size: 16 decode sequences in a 12000-block pool, one "
+                         "prefill sequence (both still larger than L2); not a bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     ws, rank, local = dist_setup()
@@ -409,7 +409,7 @@ def main():
     pw = None
     prefill_reason = None
     if want_prefill:
-        pw = PrefillWork(dev, 1239 + rank)
+        pw = PrefillWork(dev, 1239 + rank, batch=1 if args.small else 4)
         try:
             pw.append()
             pw.prefill()

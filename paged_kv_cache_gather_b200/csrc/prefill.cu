@@ -23,7 +23,9 @@
 //    (A operand in TMEM) with V as an MN-major shared-memory operand.
 //  * MMA issue order S0(j), PV1(j-1), S1(j), PV0(j): while one warpgroup
 //    turns its S into P the tensor core runs the other head's work.
-//  * K/V tiles are 128 keys: context tiles are 8 TMA boxes of 16 rows, one
+//  * K and V tiles (128 keys) have separate 2-stage rings, so the next K can
+//    land as soon as both heads' S of the current one are done, while V
+//    waits for P*V. Context tiles are 8 TMA boxes of 16 rows, one
 //    per 16-token piece of a paged block (block id from the table); chunk
 //    tiles are one 3-D box of k_new / v_new. All loads use 128-byte
 //    swizzle. Rows past the context end are loaded as out-of-bounds boxes,
@@ -48,7 +50,7 @@ constexpr int kN = 128;             // keys per tile
 constexpr int kStages = 2;          // K/V ring depth
 constexpr int kTileBytes = kN * kD * 2;   // 32 KB (K or V or Q tile)
 constexpr int kHalfBytes = kTileBytes / 2;
-constexpr int kThreads = 320;
+constexpr int kThreads = 320;       // softmax head 0 (4 warps), head 1 (4), TMA (1), MMA (1)
 constexpr int kMaxBatch = 4096;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 
@@ -83,7 +85,7 @@ struct SmemLayout {
   static constexpr int kQ1 = kTileBytes;
   static constexpr int kKV = 2 * kTileBytes;  // stage s: K at kKV + s*2*tile, V after it
   static constexpr int kBars = kKV + kStages * 2 * kTileBytes;
-  static constexpr int kNumBars = 2 + 2 * kStages + 9;
+  static constexpr int kNumBars = 2 + 4 * kStages + 9;
   static constexpr int kTmemSlot = kBars + kNumBars * 8;
   static constexpr int kQoff = kTmemSlot + 16;  // int32 [batch + 1]
   static constexpr int kMaxQt = kQoff - 8;      // int32 (placed before the prefix)
@@ -93,13 +95,15 @@ struct SmemLayout {
 enum : int {
   BAR_Q_FULL = 0,
   BAR_Q_EMPTY = 1,
-  BAR_KV_FULL = 2,                 // + stage
-  BAR_KV_EMPTY = 2 + kStages,      // + stage
-  BAR_S_FULL = 2 + 2 * kStages,    // + head
+  BAR_K_FULL = 2,                  // + stage
+  BAR_K_EMPTY = 2 + kStages,       // + stage
+  BAR_V_FULL = 2 + 2 * kStages,    // + stage
+  BAR_V_EMPTY = 2 + 3 * kStages,   // + stage
+  BAR_S_FULL = 2 + 4 * kStages,    // + head
   BAR_P_FULL = BAR_S_FULL + 2,     // + head
   BAR_O_FULL = BAR_P_FULL + 2,     // + head
   BAR_O_FREE = BAR_O_FULL + 2,     // + head
-  BAR_KV_FIXED = BAR_O_FREE + 2,   // a tile whose rows past the context end were zeroed
+  BAR_V_FIXED = BAR_O_FREE + 2,    // a V tile whose rows past the context end were zeroed
 };
 
 struct Unit {
@@ -176,12 +180,17 @@ __device__ __forceinline__ bool needs_fix(const Unit& x, bool ctx, int kp0, int 
 
 // Warp-collective bounded wait: every lane of the warp calls it and gets the
 // same answer, so the warp never splits around the warp-wide tcgen05
-// instructions that follow. On a timeout (or an abort raised by another
-// warp) it records PKV_DBG_TIMEOUT and tells every role to stop.
+// instructions that follow. With `all_lanes` false only lane 0 polls (the
+// warp's other lanes are ordered after it by the warp barrier). On a timeout
+// (or an abort raised by another warp) it records PKV_DBG_TIMEOUT and tells
+// every role to stop.
 __device__ __forceinline__ bool wait_or_flag(uint32_t bar, uint32_t parity, int32_t* dbg,
-                                             int* abort_flag) {
-  bool ok = *reinterpret_cast<volatile int*>(abort_flag) == 0 && mbar_wait(bar, parity);
+                                             int* abort_flag, bool all_lanes = false) {
+  bool ok = true;
+  if (all_lanes || (threadIdx.x & 31) == 0)
+    ok = *reinterpret_cast<volatile int*>(abort_flag) == 0 && mbar_wait(bar, parity);
   ok = __all_sync(0xffffffffu, ok);
+  __syncwarp();
   if (!ok && (threadIdx.x & 31) == 0) {
     flag_error(dbg, PKV_DBG_TIMEOUT);
     *reinterpret_cast<volatile int*>(abort_flag) = 1;
@@ -233,8 +242,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(BAR_Q_FULL), 1);
       mbar_init(bar(BAR_Q_EMPTY), 1);
       for (int s = 0; s < kStages; ++s) {
-        mbar_init(bar(BAR_KV_FULL + s), 1);
-        mbar_init(bar(BAR_KV_EMPTY + s), 1);
+        mbar_init(bar(BAR_K_FULL + s), 1);
+        mbar_init(bar(BAR_K_EMPTY + s), 1);
+        mbar_init(bar(BAR_V_FULL + s), 1);
+        mbar_init(bar(BAR_V_EMPTY + s), 1);
       }
       for (int h = 0; h < 2; ++h) {
         mbar_init(bar(BAR_S_FULL + h), 1);
@@ -242,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar(BAR_O_FULL + h), 1);
         mbar_init(bar(BAR_O_FREE + h), 128);
       }
-      mbar_init(bar(BAR_KV_FIXED), 1);
+      mbar_init(bar(BAR_V_FIXED), 1);
       *abort_flag = 0;
       fence_barrier_init();
       prefetch_tmap(&maps.q);
@@ -287,12 +298,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 8) {
     // ================================================================ TMA producer
+    const int nbox = kN / p.box_rows;  // paged boxes per context tile (8 or 16)
+    const int bs_mask = (1 << p.bs_shift) - 1;
+    // block id of this lane's box of tile j (-2: past the context end, zero fill);
+    // issued one tile ahead so the load latency hides behind the copies
+    auto fetch_id = [&](const Unit& x, int j) -> int {
+      bool ctx;
+      int idx, kp0;
+      tile_of(x, j, ctx, idx, kp0);
+      if (!ctx || lane >= nbox) return -2;
+      const int pos = kp0 + lane * p.box_rows;
+      if (pos >= x.C) return -2;
+      return p.tables[(int64_t)x.b * p.max_blocks + (pos >> p.bs_shift)];
+    };
+    // row of a paged box, or the first out-of-bounds row (TMA fills zeros)
+    auto box_row = [&](const Unit& x, int id, int pos) -> int {
+      if (id == -2) return p.pool_rows;
+      if (id < 0 || id >= p.num_blocks) {
+        flag_error(p.dbg, PKV_DBG_BLOCK_ID);
+        return p.pool_rows;
+      }
+      return ((id * p.num_kv_heads + x.kvh) << p.bs_shift) + (pos & bs_mask);
+    };
     int unit_k = 0;
-    uint32_t kv_count = 0;
+    uint32_t cnt = 0;  // tiles issued (K and V rings advance together)
     for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
       const Unit x = unit_of(p, qoff, max_qt, u);
       if (!x.valid) continue;
       const int h0 = x.kvh * p.group + x.hp * (p.two_heads ? 2 : 1);
+      const int n = x.n();
+      int id_cur = fetch_id(x, 0);
       // query tiles (slot reusable once the previous unit's MMAs are done)
       if (unit_k > 0 && !wait_or_flag(bar(BAR_Q_EMPTY), (unit_k - 1) & 1, p.dbg, abort_flag)) break;
       if (lane == 0) {
@@ -303,92 +338,64 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(smem_u32(smem + (hh ? L::kQ1 : L::kQ0) + half * kHalfBytes), &maps.q,
                         half * 64, h0 + hh, row0, bar(BAR_Q_FULL));
       }
-      // key/value tiles
-      const int n = x.n();
-      for (int j = 0; j < n; ++j, ++kv_count) {
-        const int s = kv_count % kStages;
-        if (kv_count >= (uint32_t)kStages &&
-            !wait_or_flag(bar(BAR_KV_EMPTY + s), ((kv_count / kStages) - 1) & 1, p.dbg,
-                          abort_flag))
-          break;
+      bool ok = true;
+      for (int j = 0; j < n; ++j, ++cnt) {
+        const int s = cnt % kStages;
+        const uint32_t ph = ((cnt / kStages) - 1) & 1;
         bool ctx;
         int idx, kp0;
         tile_of(x, j, ctx, idx, kp0);
+        const int id_next = (j + 1 < n) ? fetch_id(x, j + 1) : -2;
         const uint32_t kdst = smem_u32(smem + L::kKV + s * 2 * kTileBytes);
         const uint32_t vdst = kdst + kTileBytes;
-        const uint32_t fb = bar(BAR_KV_FULL + s);
-        if (lane == 0) mbar_arrive_expect_tx(fb, 2 * kTileBytes);
-        __syncwarp();
-        if (!ctx) {
-          if (lane == 0) {
-            const int row0 = x.qoff + idx * kN;
-            for (int half = 0; half < 2; ++half) {
-              tma_load_3d(kdst + half * kHalfBytes, &maps.knew, half * 64, x.kvh, row0, fb);
-              tma_load_3d(vdst + half * kHalfBytes, &maps.vnew, half * 64, x.kvh, row0, fb);
-            }
+        for (int kv = 0; kv < 2; ++kv) {
+          const uint32_t dst = kv ? vdst : kdst;
+          const uint32_t fb = bar((kv ? BAR_V_FULL : BAR_K_FULL) + s);
+          if (cnt >= (uint32_t)kStages &&
+              !wait_or_flag(bar((kv ? BAR_V_EMPTY : BAR_K_EMPTY) + s), ph, p.dbg, abort_flag)) {
+            ok = false;
+            break;
           }
-        } else {
-          // one lane per box of `box_rows` paged rows
-          const int nbox = kN / p.box_rows;
-          for (int bi = lane; bi < nbox; bi += 32) {
-            const int pos = kp0 + bi * p.box_rows;
-            const uint32_t off = bi * p.box_rows * 128;
-            if (pos + p.box_rows <= x.C) {
-              const int j_blk = pos >> p.bs_shift;
-              int id = p.tables[(int64_t)x.b * p.max_blocks + j_blk];
-              int row;
-              if (id < 0 || id >= p.num_blocks) {
-                flag_error(p.dbg, PKV_DBG_BLOCK_ID);
-                row = p.pool_rows;  // out of bounds: zero fill
-              } else {
-                row = ((id * p.num_kv_heads + x.kvh) << p.bs_shift) + (pos & ((1 << p.bs_shift) - 1));
-              }
-              for (int half = 0; half < 2; ++half) {
-                tma_load_2d(kdst + half * kHalfBytes + off, &maps.kpool, half * 64, row, fb);
-                tma_load_2d(vdst + half * kHalfBytes + off, &maps.vpool, half * 64, row, fb);
-              }
-            } else if (pos >= x.C) {
-              for (int half = 0; half < 2; ++half) {
-                tma_load_2d(kdst + half * kHalfBytes + off, &maps.kpool, half * 64, p.pool_rows, fb);
-                tma_load_2d(vdst + half * kHalfBytes + off, &maps.vpool, half * 64, p.pool_rows, fb);
-              }
-            } else {
-              // straddles the context end: load the block; rows past the end are
-              // zeroed below once the tile has landed
-              const int j_blk = pos >> p.bs_shift;
-              int id = p.tables[(int64_t)x.b * p.max_blocks + j_blk];
-              int row;
-              if (id < 0 || id >= p.num_blocks) {
-                flag_error(p.dbg, PKV_DBG_BLOCK_ID);
-                row = p.pool_rows;
-              } else {
-                row = ((id * p.num_kv_heads + x.kvh) << p.bs_shift) + (pos & ((1 << p.bs_shift) - 1));
-              }
-              for (int half = 0; half < 2; ++half) {
-                tma_load_2d(kdst + half * kHalfBytes + off, &maps.kpool, half * 64, row, fb);
-                tma_load_2d(vdst + half * kHalfBytes + off, &maps.vpool, half * 64, row, fb);
-              }
+          if (lane == 0) mbar_arrive_expect_tx(fb, kTileBytes);
+          __syncwarp();
+          if (!ctx) {
+            if (lane == 0) {
+              const int row0 = x.qoff + idx * kN;
+              for (int half = 0; half < 2; ++half)
+                tma_load_3d(dst + half * kHalfBytes, kv ? &maps.vnew : &maps.knew, half * 64,
+                            x.kvh, row0, fb);
             }
-          }
-          if (needs_fix(x, ctx, kp0, p.box_rows)) {
-            if (!wait_or_flag(fb, (kv_count / kStages) & 1, p.dbg, abort_flag)) break;
-            // zero V rows [C - kp0, end of that box) in both 64-column halves
-            const int r0 = x.C - kp0;
-            const int r1 = (r0 / p.box_rows + 1) * p.box_rows;
-            uint8_t* vbase = smem + L::kKV + s * 2 * kTileBytes + kTileBytes;
-            for (int i = lane; i < (r1 - r0) * 2 * 8; i += 32) {
-              const int rr = r0 + i / 16;
-              const int half = (i / 8) & 1;
-              const int ch = i & 7;
-              *reinterpret_cast<int4*>(vbase + half * kHalfBytes + rr * 128 + ch * 16) =
-                  make_int4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(BAR_KV_FIXED));
+          } else if (lane < nbox) {
+            const int pos = kp0 + lane * p.box_rows;
+            const int row = box_row(x, id_cur, pos);
+            const uint32_t off = lane * p.box_rows * 128;
+            for (int half = 0; half < 2; ++half)
+              tma_load_2d(dst + half * kHalfBytes + off, kv ? &maps.vpool : &maps.kpool,
+                          half * 64, row, fb);
           }
         }
+        if (!ok) break;
+        if (needs_fix(x, ctx, kp0, p.box_rows)) {
+          // the box holding the context end also holds pool rows past it:
+          // zero them in V once the tile has landed, then release the MMA warp
+          if (!wait_or_flag(bar(BAR_V_FULL + s), (cnt / kStages) & 1, p.dbg, abort_flag)) break;
+          const int r0 = x.C - kp0;
+          const int r1 = (r0 / p.box_rows + 1) * p.box_rows;
+          uint8_t* vbase = smem + L::kKV + s * 2 * kTileBytes + kTileBytes;
+          for (int i = lane; i < (r1 - r0) * 2 * 8; i += 32) {
+            const int rr = r0 + i / 16;
+            const int half = (i / 8) & 1;
+            const int ch = i & 7;
+            *reinterpret_cast<int4*>(vbase + half * kHalfBytes + rr * 128 + ch * 16) =
+                make_int4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_V_FIXED));
+        }
+        id_cur = id_next;
       }
+      if (!ok) break;
       ++unit_k;
     }
   } else if (warp == 9) {
@@ -398,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t S0 = tmem, S1 = tmem + 128, O0 = tmem + 256, O1 = tmem + 384;
     const uint32_t q0 = smem_u32(smem + L::kQ0), q1 = smem_u32(smem + L::kQ1);
     int unit_k = 0;
-    uint32_t kv_count = 0, p_cnt0 = 0, p_cnt1 = 0, fix_count = 0;
+    uint32_t cnt = 0, p_cnt0 = 0, p_cnt1 = 0, fix_count = 0;
     auto issue_s = [&](uint32_t d, uint32_t qa, uint32_t ka) {
 #pragma unroll
       for (int kk = 0; kk < kD / 16; ++kk) {
@@ -420,30 +427,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n = x.n();
       if (!wait_or_flag(bar(BAR_Q_FULL), unit_k & 1, p.dbg, abort_flag)) break;
       tc::fence_after_sync();
-      uint32_t prev_v = 0;
       int prev_s = 0;
       bool ok = true;
-      for (int j = 0; j < n && ok; ++j, ++kv_count) {
-        const int s = kv_count % kStages;
-        if (!wait_or_flag(bar(BAR_KV_FULL + s), (kv_count / kStages) & 1, p.dbg, abort_flag)) {
-          ok = false;
-          break;
-        }
-        {
-          bool ctx_t;
-          int idx_t, kp0_t;
-          tile_of(x, j, ctx_t, idx_t, kp0_t);
-          if (needs_fix(x, ctx_t, kp0_t, p.box_rows)) {
-            if (!wait_or_flag(bar(BAR_KV_FIXED), fix_count & 1, p.dbg, abort_flag)) {
-              ok = false;
-              break;
-            }
-            ++fix_count;
-          }
-        }
-        tc::fence_after_sync();
+      for (int j = 0; j < n; ++j, ++cnt) {
+        const int s = cnt % kStages;
+        const uint32_t ph = (cnt / kStages) & 1;
         const uint32_t ka = smem_u32(smem + L::kKV + s * 2 * kTileBytes);
         const uint32_t va = ka + kTileBytes;
+        if (!(ok = wait_or_flag(bar(BAR_K_FULL + s), ph, p.dbg, abort_flag))) break;
+        tc::fence_after_sync();
         if (lane == 0) {
           issue_s(S0, q0, ka);
           tc::commit(bar(BAR_S_FULL + 0));
@@ -451,14 +443,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (p.two_heads) {
           if (j > 0) {
-            if (!wait_or_flag(bar(BAR_P_FULL + 1), p_cnt1 & 1, p.dbg, abort_flag)) { ok = false; break; }
+            if (!(ok = wait_or_flag(bar(BAR_P_FULL + 1), p_cnt1 & 1, p.dbg, abort_flag))) break;
             ++p_cnt1;
+            if (j == 1 && unit_k > 0 &&
+                !(ok = wait_or_flag(bar(BAR_O_FREE + 1), (unit_k - 1) & 1, p.dbg, abort_flag)))
+              break;
             tc::fence_after_sync();
-            if (j - 1 == 0 && unit_k > 0 &&
-                !wait_or_flag(bar(BAR_O_FREE + 1), (unit_k - 1) & 1, p.dbg, abort_flag)) { ok = false; break; }
             if (lane == 0) {
-              issue_pv(O1, S1, prev_v, j - 1 > 0);
-              tc::commit(bar(BAR_KV_EMPTY + prev_s));
+              issue_pv(O1, S1, smem_u32(smem + L::kKV + prev_s * 2 * kTileBytes) + kTileBytes,
+                       j - 1 > 0);
+              tc::commit(bar(BAR_V_EMPTY + prev_s));
             }
             __syncwarp();
           }
@@ -468,29 +462,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __syncwarp();
         }
-        if (!wait_or_flag(bar(BAR_P_FULL + 0), p_cnt0 & 1, p.dbg, abort_flag)) { ok = false; break; }
+        if (lane == 0) tc::commit(bar(BAR_K_EMPTY + s));  // K of this tile is no longer read
+        __syncwarp();
+        if (!(ok = wait_or_flag(bar(BAR_V_FULL + s), ph, p.dbg, abort_flag))) break;
+        {
+          bool ctx_t;
+          int idx_t, kp0_t;
+          tile_of(x, j, ctx_t, idx_t, kp0_t);
+          if (needs_fix(x, ctx_t, kp0_t, p.box_rows)) {
+            if (!(ok = wait_or_flag(bar(BAR_V_FIXED), fix_count & 1, p.dbg, abort_flag))) break;
+            ++fix_count;
+          }
+        }
+        if (!(ok = wait_or_flag(bar(BAR_P_FULL + 0), p_cnt0 & 1, p.dbg, abort_flag))) break;
         ++p_cnt0;
-        tc::fence_after_sync();
         if (j == 0 && unit_k > 0 &&
-            !wait_or_flag(bar(BAR_O_FREE + 0), (unit_k - 1) & 1, p.dbg, abort_flag)) { ok = false; break; }
+            !(ok = wait_or_flag(bar(BAR_O_FREE + 0), (unit_k - 1) & 1, p.dbg, abort_flag)))
+          break;
+        tc::fence_after_sync();
         if (lane == 0) {
           issue_pv(O0, S0, va, j > 0);
-          if (!p.two_heads) tc::commit(bar(BAR_KV_EMPTY + s));
+          if (!p.two_heads) tc::commit(bar(BAR_V_EMPTY + s));
         }
         __syncwarp();
-        prev_v = va;
         prev_s = s;
       }
       if (!ok) break;
       if (p.two_heads) {
         if (!wait_or_flag(bar(BAR_P_FULL + 1), p_cnt1 & 1, p.dbg, abort_flag)) break;
         ++p_cnt1;
-        tc::fence_after_sync();
         if (n == 1 && unit_k > 0 &&
-            !wait_or_flag(bar(BAR_O_FREE + 1), (unit_k - 1) & 1, p.dbg, abort_flag)) break;
+            !wait_or_flag(bar(BAR_O_FREE + 1), (unit_k - 1) & 1, p.dbg, abort_flag))
+          break;
+        tc::fence_after_sync();
         if (lane == 0) {
-          issue_pv(O1, S1, prev_v, n - 1 > 0);
-          tc::commit(bar(BAR_KV_EMPTY + prev_s));
+          issue_pv(O1, S1, smem_u32(smem + L::kKV + prev_s * 2 * kTileBytes) + kTileBytes,
+                   n - 1 > 0);
+          tc::commit(bar(BAR_V_EMPTY + prev_s));
         }
         __syncwarp();
       }
@@ -502,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       ++unit_k;
     }
-  } else {
+  } else if (warp < 8) {
     // ================================================================ softmax warpgroups
     const int hsel = warp >> 2;              // which head of the pair
     const int row = (warp & 3) * 32 + lane;  // query row of the tile = TMEM lane
@@ -525,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < n; ++j, ++s_cnt) {
-        if (!wait_or_flag(bar(BAR_S_FULL + hsel), s_cnt & 1, p.dbg, abort_flag)) { ok = false; break; }
+        if (!wait_or_flag(bar(BAR_S_FULL + hsel), s_cnt & 1, p.dbg, abort_flag, true)) { ok = false; break; }
         tc::fence_after_sync();
         bool ctx;
         int idx, kp0;
@@ -534,26 +542,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool full = kp0 + kN <= key_end;
         if (p.mask_kind != PKV_MASK_NONE) full = full && (kp0 + kN - 1 <= qmin);
         if (x.window > 0) full = full && (qmax - kp0 < x.window);
-        // pass 1: row maximum over the visible keys of the tile
-        float mx = -INFINITY;
+        // pass 1: the whole S row of this thread in one tensor-memory round trip
+        float mx;
+        {
+          uint32_t r[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tc::ld32(S + c * 32, r);
+          for (int c = 0; c < 4; ++c) tc::ld32(S + c * 32, r[c]);
           tc::wait_ld();
-          if (full) {
+          if (!full) {
+            // the visible keys of a row form one interval of columns [vlo, vhi);
+            // masked scores become -inf in tensor memory, so pass 2 needs no mask
+            int vhi = min(kN, key_end - kp0), vlo = 0;
+            if (p.mask_kind != PKV_MASK_NONE) vhi = min(vhi, qpos - kp0 + 1);
+            if (x.window > 0) vlo = max(0, qpos - x.window + 1 - kp0);
+            const uint32_t span = (uint32_t)max(vhi - vlo, 0);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(r[i]));
-          } else {
+            for (int c = 0; c < 4; ++c) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int kpos = kp0 + c * 32 + i;
-              bool vis = kpos < key_end;
-              if (p.mask_kind != PKV_MASK_NONE) vis = vis && kpos <= qpos;
-              if (x.window > 0) vis = vis && (qpos - kpos < x.window);
-              if (vis) mx = fmaxf(mx, __uint_as_float(r[i]));
+              for (int i = 0; i < 32; ++i)
+                if ((uint32_t)(c * 32 + i - vlo) >= span) r[c][i] = __float_as_uint(-INFINITY);
+              tc::st32(S + c * 32, r[c]);
             }
+            tc::wait_st();
           }
+          float mx4[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float a0 = __uint_as_float(r[c][0]), a1 = __uint_as_float(r[c][1]);
+#pragma unroll
+            for (int i = 2; i < 32; i += 2) {
+              a0 = fmaxf(a0, __uint_as_float(r[c][i]));
+              a1 = fmaxf(a1, __uint_as_float(r[c][i + 1]));
+            }
+            mx4[c] = fmaxf(a0, a1);
+          }
+          mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
         }
         const float mxs = mx * p.scale_log2;  // scale > 0 keeps the order
         // lazy rescale: move the reference maximum only when it grows by > 2^8
@@ -563,43 +586,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = mxs;
         }
         const float mb = (m == -INFINITY) ? 0.f : m;
-        float ls0 = 0.f, ls1 = 0.f;
-        // pass 2: P = exp2(s*c - m) (0 for masked keys), bf16 into the S columns
+        // pass 2, two halves of 64 columns: P = exp2(s*c - m) (masked -inf -> 0),
+        // packed in place to bf16 pairs (P[2k], P[2k+1] -> word k), stored over
+        // the first 64 columns of S
+        float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-          uint32_t r0[32], r1[32], pk[32];
-          tc::ld32(S + hf * 64, r0);
-          tc::ld32(S + hf * 64 + 32, r1);
+          uint32_t r[2][32];
+          tc::ld32(S + hf * 64, r[0]);
+          tc::ld32(S + hf * 64 + 32, r[1]);
           tc::wait_ld();
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              const float s0 = __uint_as_float(cc ? r1[i] : r0[i]);
-              const float s1 = __uint_as_float(cc ? r1[i + 1] : r0[i + 1]);
-              float e0 = fast_exp2(fmaf(s0, p.scale_log2, -mb));
-              float e1 = fast_exp2(fmaf(s1, p.scale_log2, -mb));
-              if (!full) {
-                const int kpos = kp0 + hf * 64 + cc * 32 + i;
-                bool v0 = kpos < key_end, v1 = kpos + 1 < key_end;
-                if (p.mask_kind != PKV_MASK_NONE) {
-                  v0 = v0 && kpos <= qpos;
-                  v1 = v1 && kpos + 1 <= qpos;
-                }
-                if (x.window > 0) {
-                  v0 = v0 && (qpos - kpos < x.window);
-                  v1 = v1 && (qpos - kpos - 1 < x.window);
-                }
-                e0 = v0 ? e0 : 0.f;
-                e1 = v1 ? e1 : 0.f;
-              }
-              ls0 += e0;
-              ls1 += e1;
-              pk[cc * 16 + i / 2] = pack_bf16x2(e0, e1);
+            for (int i = 0; i < 32; ++i) {
+              const float e = fast_exp2(fmaf(__uint_as_float(r[c][i]), p.scale_log2, -mb));
+              ls[i & 7] += e;
+              r[c][i] = __float_as_uint(e);
             }
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const int f0 = 2 * k, f1 = 2 * k + 1;
+            r[0][k] = pack_bf16x2(__uint_as_float(r[f0 >> 5][f0 & 31]),
+                                  __uint_as_float(r[f1 >> 5][f1 & 31]));
           }
-          tc::st32(S + hf * 32, pk);
+          tc::st32(S + hf * 32, r[0]);
         }
+        const float ls0 = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        const float ls1 = (ls[4] + ls[5]) + (ls[6] + ls[7]);
         l = l * alpha + ls0 + ls1;
         // tcgen05.ld/st are warp-collective: the whole warp takes this branch
         // when any of its rows moved its maximum (the others scale by 1)
@@ -622,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16, lse
-      if (!wait_or_flag(bar(BAR_O_FULL + hsel), unit_k & 1, p.dbg, abort_flag)) break;
+      if (!wait_or_flag(bar(BAR_O_FULL + hsel), unit_k & 1, p.dbg, abort_flag, true)) break;
       tc::fence_after_sync();
       const int h = x.kvh * p.group + x.hp * (p.two_heads ? 2 : 1) + hsel;
       const bool valid_row = i_row < x.Q && x.qoff + i_row < p.total_q;
