@@ -258,6 +258,100 @@ class PrefillWork:
         self.lse_h.copy_(self.lse, non_blocking=True)
 
 
+# ------------------------------------------------------------------ side measurements
+
+def l2_flush_buffer(dev):
+    return torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+
+def time_calls(fn, n, flush=None, stream=None):
+    """Mean device time of fn() over n calls (CUDA events on the launching
+    stream); when `flush` is given it is overwritten before every call, outside
+    the event pair, so each call starts with a cold L2."""
+    stream = stream or torch.cuda.current_stream()
+    ts = []
+    for _ in range(n):
+        if flush is not None:
+            flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return sum(ts) / len(ts)
+
+
+def decode_sweep(dev, flush):
+    """Batch-1 decode over 128..4096 tokens (32/8 heads, d 128, causal), the
+    shape of the pages' sequence-length sweep: microseconds per call with a cold
+    L2, eagerly and as a replayed CUDA graph, and the 2048/128 latency ratio."""
+    import paged_kv_cache_gather_b200 as pkv
+    from paged_kv_cache_gather_b200 import inputs as I
+
+    base = I.config2(4096)
+    kc, vc = base.k_cache.to(dev), base.v_cache.to(dev)
+    q = base.q.to(dev)
+    res = {}
+    for L in I.CONFIG2_LENGTHS:
+        tab = base.block_tables[:, : L // 16].contiguous().to(dev)
+        lens = torch.tensor([L], dtype=torch.int32, device=dev)
+        out = torch.empty_like(q)
+        lse = torch.empty(1, 32, dtype=torch.float32, device=dev)
+        ws = pkv.decode_workspace(1, 32, kc)
+        mask = pkv.causal()
+        call = lambda: pkv.paged_attention_decode(q, kc, vc, tab, lens, base.scale, mask,
+                                                  out=out, lse=lse, workspace=ws)
+        for _ in range(3):
+            call()
+        eager = time_calls(call, 20, flush)
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            call()
+        torch.cuda.current_stream().wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call()
+        graph = time_calls(g.replay, 20, flush)
+        kv = L * 8 * 128 * 2 * 2
+        res[str(L)] = {"us_eager": round(eager * 1e3, 2), "us_graph": round(graph * 1e3, 2),
+                       "kv_GBps_graph": round(kv / (graph * 1e-3) / 1e9, 1)}
+    res["latency_ratio_2048_over_128"] = round(res["2048"]["us_graph"] / res["128"]["us_graph"], 2)
+    res["pages_ratio_on_L4"] = "about 2x, end to end in a model (context only)"
+    return res
+
+
+def shared_prefix(dev, flush):
+    """8 groups x 8 beams, 4096-token prefix shared by block id + 256 own tokens:
+    decode time with shared blocks and with copied ones; logical bytes are what
+    the beams read, unique bytes what is stored."""
+    import paged_kv_cache_gather_b200 as pkv
+    from paged_kv_cache_gather_b200 import inputs as I
+
+    out = {}
+    for shared in (True, False):
+        c = I.config4(shared=shared)
+        kc, vc = c.k_cache.to(dev), c.v_cache.to(dev)
+        q, tab, lens = c.q.to(dev), c.block_tables.to(dev), c.seq_lens.to(dev)
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=dev)
+        ws = pkv.decode_workspace(q.shape[0], q.shape[1], kc)
+        call = lambda: pkv.paged_attention_decode(q, kc, vc, tab, lens, c.scale, pkv.causal(),
+                                                  out=o, lse=lse, workspace=ws)
+        for _ in range(3):
+            call()
+        ms = time_calls(call, 20, flush)
+        logical = 64 * 4352 * 8 * 128 * 2 * 2
+        unique = c.extra["unique_blocks"] * 8 * 16 * 128 * 2 * 2
+        out["shared" if shared else "copied"] = {
+            "us": round(ms * 1e3, 2), "logical_GBps": round(logical / (ms * 1e-3) / 1e9, 1),
+            "unique_bytes": unique, "unique_GBps": round(unique / (ms * 1e-3) / 1e9, 1)}
+        del kc, vc
+        torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------------ CPU baseline
 
 def oracle_decode_sample(budget_s=12.0, seed=None):
@@ -321,16 +415,20 @@ def cpu_threads():
 
 # ------------------------------------------------------------------ main
 
-def dist_setup():
+def dist_setup(backend="nccl"):
+    """One process per GPU (torchrun env vars); returns (world size, rank, local rank)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if ws > 1:
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
     return ws, rank, local
 
 
@@ -351,27 +449,55 @@ def max_over_ranks(x, ws, dev):
     return float(t.item())
 
 
+def workload_config(with_prefill, ws):
+    return {
+        "workload": ("ragged batched decode (64 seqs, lengths U[1,8192] growing 1/step, 32/8 "
+                     "heads, d128, bf16, block 16, 40000-block shuffled pool, window 4096 on even "
+                     "seqs)" + (" + chunked prefill (4 x (30720 ctx + 2048 chunk), causal)"
+                                if with_prefill else "")),
+        "l2": "inputs larger than L2: 0.86 GB of KV per decode step, 537 MB per prefill step "
+              "(126 MB L2), no flush",
+        "parallelism": f"replicas x{ws} (independent batches, no collective)"}
+
+
 def run_reference(args, ws, rank):
+    """The float64 CPU oracle as it stands, on whole decode steps of the same
+    ragged batch (one step = all 64 sequences x 32 heads)."""
     if rank != 0:
         return
-    pk, _ = peaks()
-    samples = []
-    for _ in range(args.warmup):
-        oracle_decode_sample(budget_s=0.0)
+    import oracle
+    from paged_kv_cache_gather_b200 import inputs as I
+
+    c = I.config3()
+    vis = visible_tokens(c.seq_lens.numpy(), c.window_per_seq.numpy())
+    per_step = 8  # sequences per reference step: a bounded sample, cycling through the batch
+    done = {"bytes": 0.0}
+
+    def step(k):
+        seqs = [(8 * k + i) % c.batch for i in range(per_step)]
+        rows = [(b, h) for b in seqs for h in range(c.num_q_heads)]
+        oracle.paged_decode_rows(c.q, c.k_cache, c.v_cache, c.block_tables, c.seq_lens, c.scale,
+                                 c.mask_kind, c.window, c.window_per_seq, rows=rows)
+        return float(vis[seqs].sum() * c.num_kv_heads * c.head_dim * 2 * 2)
+
+    for k in range(args.warmup):
+        step(k)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        samples.append(oracle_decode_sample(budget_s=0.0))
+    total = 0.0
+    for k in range(args.steps):
+        total += step(args.warmup + k)
     el = time.perf_counter() - t0
-    val = statistics.mean(s["value"] for s in samples)
+    val = total / el / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(el * 1e3 / max(args.steps, 1), 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "ragged batched decode: 64 seqs, lengths U[1,8192], 32/8 heads, "
-                                   "d128, bf16 pools, block 16, window 4096 on even seqs"},
+            "config": workload_config(args.workload in ("all", "prefill"), 1),
             "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": cpu_threads(),
                              "kind": "oracle",
-                             "sample": "one full decode step of the ragged batch per step"},
+                             "sample": "8 sequences x 32 heads of the ragged batch per step, "
+                                       "cycling through the batch; float64 NumPy, inputs "
+                                       "generated once"},
             "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -385,6 +511,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="all", choices=["all", "decode", "prefill"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the batch-1 sweep and the shared-prefix measurement")
     ap.add_argument("--small", action="store_true",
                     help="profiling size: 16 decode sequences in a 12000-block pool, one "
                          "prefill sequence (both still larger than L2); not a bench line")
@@ -540,14 +668,13 @@ def main():
         line.update({"value": line["prefill"]["value"], "unit": "TFLOP/s",
                      "roofline": line["prefill"]["roofline"], "e2e": line["prefill"]["e2e"]})
     line["gpu_launches"] = launches
-    line["config"] = {
-        "workload": ("ragged batched decode (64 seqs, lengths U[1,8192] growing 1/step, 32/8 heads, "
-                     "d128, bf16, block 16, 40000-block shuffled pool, window 4096 on even seqs)"
-                     + (" + chunked prefill (4 x (30720 ctx + 2048 chunk), causal)" if pw else "")),
-        "l2": "inputs larger than L2: 0.94 GB of KV per decode step, 537 MB per prefill step "
-              "(126 MB L2), no flush",
-        "parallelism": f"replicas x{ws} (independent batches, no collective)"}
+    line["config"] = workload_config(pw is not None, ws)
     line["clocks"] = clk
+    if rank == 0 and not args.no_extras and not args.small and want_decode:
+        flush = l2_flush_buffer(dev)
+        line["decode_sweep_batch1"] = decode_sweep(dev, flush)
+        line["shared_prefix_beams"] = shared_prefix(dev, flush)
+        del flush
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_decode_sample()
         if pw:
