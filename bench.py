@@ -50,6 +50,37 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+# ------------------------------------------------------------------ profiled traffic
+
+# DRAM bytes (read + write) per unit of work, from one ncu capture of each
+# kernel on a smaller case of the same workload (profiles/*.md); a full launch
+# scales it by its units. Valid only for the kernel sources it was taken on:
+# after any change to them the bench reports null until they are profiled again.
+PROFILED_TRAFFIC = {
+    "decode": {"sources": ['csrc/decode.cu', 'csrc/pkv_common.cuh'],
+               "sha256": "f1968cf1c3212cc986b1c73324cfd7316f253afe4c997a4d72fd254c89b61551",
+               "per_unit": 194937344 / 190134992,  # per algorithmic byte (16-seq ragged case)
+               },
+    "prefill": {"sources": ['csrc/prefill.cu', 'csrc/pkv_common.cuh', 'csrc/tc_sm100.cuh'],
+                "sha256": "4dc33d68e9819d7d3630fa72963d01a2e87df90a997ea37017c996f5990e4372",
+                "per_unit": 299044608 / 1065168666624,  # per causal FLOP (1-seq case)
+                },
+}
+
+
+def profiled_traffic(kind, units):
+    import hashlib
+
+    rec = PROFILED_TRAFFIC[kind]
+    h = hashlib.sha256()
+    for f in rec["sources"]:
+        with open(os.path.join(ROOT, "paged_kv_cache_gather_b200", f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != rec["sha256"]:
+        return None
+    return int(rec["per_unit"] * units)
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -633,7 +664,8 @@ def main():
             "roofline": {"kernel": "paged_attention_decode (main + combine)", "bound": "hbm",
                          "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": round(achieved / pk["hbm_gbs"], 4),
-                         "peak_kind": pk_kind, "traffic": None,
+                         "peak_kind": pk_kind,
+                         "traffic": profiled_traffic("decode", (kv + io) / n),
                          "bytes_per_launch": int((kv + io) / n)},
             "e2e": {"value": round(kv * ws / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": int(dw.h2d), "d2h_bytes_per_step": int(dw.d2h)},
@@ -657,7 +689,8 @@ def main():
                          "achieved": round(tf, 1), "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": round(tf / peak_tf, 4),
                          "frac_of_sustained": round(tf / pk.get("bf16_tflops_sustained", peak_tf), 4),
-                         "peak_kind": pk_kind, "traffic": None},
+                         "peak_kind": pk_kind,
+                         "traffic": profiled_traffic("prefill", pw.flops)},
             "e2e": {"value": round(pw.flops * n * ws / (pe2e * 1e-3) / 1e12, 2),
                     "unit": "TFLOP/s", "h2d_bytes_per_step": int(pw.h2d),
                     "d2h_bytes_per_step": int(pw.d2h)}}
