@@ -216,6 +216,14 @@ PKV_API int paged_attention_decode_noalloc(const void* q, const void* k_cache, c
                                            pkv_mask_mod mask, void* out, float* lse,
                                            int32_t* dbg_err, void* stream);
 
+/*
+ * pkv_debug_exp2 — diagnostic, not part of the attention API: y[i] = 2^x[i]
+ * computed by the FMA-pipe exponential the prefill softmax uses for part of its
+ * elements (exact base-2 range reduction plus a fitted cubic; relative error
+ * <= 1e-4 for -126 <= x <= 127, exactly 0 below -126). x, y: device float32 [n].
+ */
+PKV_API int pkv_debug_exp2(const float* x, float* y, int32_t n, void* stream);
+
 /* Name of a status code (static string). */
 PKV_API const char* pkv_status_string(int status);
 

@@ -39,6 +39,7 @@ EXPORTS = (
     "paged_attention_decode",
     "paged_attention_prefill",
     "paged_attention_decode_noalloc",
+    "pkv_debug_exp2",
     "pkv_status_string",
     "pkv_last_error",
     "pkv_version",
@@ -89,6 +90,8 @@ def _declare(lib):
     lib.paged_attention_decode_noalloc.argtypes = [_vp, _vp, _vp, CacheDescC, _vp, _i32, _vp, _i32,
                                                    _i32, _f32, MaskModC, _vp, _vp, _vp, _vp]
     lib.paged_attention_decode_noalloc.restype = ctypes.c_int
+    lib.pkv_debug_exp2.argtypes = [_vp, _vp, _i32, _vp]
+    lib.pkv_debug_exp2.restype = ctypes.c_int
     lib.pkv_status_string.argtypes = [ctypes.c_int]
     lib.pkv_status_string.restype = ctypes.c_char_p
     lib.pkv_last_error.argtypes = []

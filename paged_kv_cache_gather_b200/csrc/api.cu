@@ -8,6 +8,7 @@
 
 #include <mutex>
 
+#include "pkv_common.cuh"
 #include "pkv_internal.h"
 
 namespace pkv {
@@ -234,6 +235,20 @@ int paged_attention_prefill(const void* q, const void* k_new, const void* v_new,
                 ctx_lens, q_lens, batch, total_q, num_q_heads, scale, mask, out,
                 lse,      dbg_err, static_cast<cudaStream_t>(stream)};
   return launch_prefill(a);
+}
+
+__global__ void debug_exp2_kernel(const float* x, float* y, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    y[i] = exp2_fma(x[i]);
+}
+
+int pkv_debug_exp2(const float* x, float* y, int32_t n, void* stream) {
+  g_last_error[0] = 0;
+  if (n < 0 || (n > 0 && (!x || !y))) return fail(PKV_ERR_INVALID_ARG, "pkv_debug_exp2: bad args");
+  if (n == 0) return PKV_OK;
+  debug_exp2_kernel<<<(n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184, 256, 0,
+                      static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return check_launch("pkv_debug_exp2");
 }
 
 }  // extern "C"

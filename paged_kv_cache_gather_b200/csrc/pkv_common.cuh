@@ -154,6 +154,52 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Packed float pairs (Blackwell f32x2 arithmetic): one instruction, two lanes.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// max of three floats in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x on the FMA pipe, for x <= 127 (used for part of the softmax exponentials
+// so the MUFU unit is not the only one doing them). Exact base-2 range
+// reduction x = j + f, j = round(x) (via the 1.5*2^23 rounding constant),
+// f in [-1/2, 1/2]; 2^f by a cubic fitted for minimum relative error
+// (paged_kv_cache_gather_b200/fit_exp2.py: max relative error 7.5e-5, 1.0e-4
+// along this float32 path); j is added to the exponent field. x < -126
+// (including -inf) gives exactly 0.
+__device__ __forceinline__ float exp2_fma(float x) {
+  const float magic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+  const float xc = fmaxf(x, -126.0f);
+  const float t = xc + magic;
+  const float j = t - magic;
+  const float f = xc - j;
+  float p = fmaf(5.517132208e-02f, f, 2.426105440e-01f);
+  p = fmaf(p, f, 6.932609677e-01f);
+  p = fmaf(p, f, 9.999281168e-01f);
+  const int bits = __float_as_int(p) + (__float_as_int(t) << 23);
+  return x < -126.0f ? 0.0f : __int_as_float(bits);
+}
+
 __device__ __forceinline__ void flag_error(int32_t* dbg, int32_t bit) {
   if (dbg) atomicOr(dbg, bit);
 }

@@ -406,20 +406,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t q0 = smem_u32(smem + L::kQ0), q1 = smem_u32(smem + L::kQ1);
     int unit_k = 0;
     uint32_t cnt = 0, p_cnt0 = 0, p_cnt1 = 0, fix_count = 0;
-    auto issue_s = [&](uint32_t d, uint32_t qa, uint32_t ka) {
+    // Descriptors are built once; the k-steps only move the start address
+    // (16-byte units in the low bits): +2 per 32-byte step inside a 128-byte
+    // swizzle row, +1024 per 64-column half (16 KB), +128 per 16 V rows.
+    const uint64_t dq0 = tc::smem_desc(q0, 16, 1024, tc::kSwizzle128B);
+    const uint64_t dq1 = tc::smem_desc(q1, 16, 1024, tc::kSwizzle128B);
+    const uint64_t dk0 = tc::smem_desc(smem_u32(smem + L::kKV), 16, 1024, tc::kSwizzle128B);
+    const uint64_t dv0 =
+        tc::smem_desc(smem_u32(smem + L::kKV) + kTileBytes, kHalfBytes, 1024, tc::kSwizzle128B);
+    constexpr uint64_t kStageStep = (uint64_t)(2 * kTileBytes) >> 4;
+    auto issue_s = [&](uint32_t d, uint64_t dq, uint64_t dk) {
 #pragma unroll
       for (int kk = 0; kk < kD / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-        tc::mma_ss(d, tc::smem_desc(qa + off, 16, 1024, tc::kSwizzle128B),
-                   tc::smem_desc(ka + off, 16, 1024, tc::kSwizzle128B), idesc_s, kk > 0);
+        const uint64_t off = (uint64_t)((kk >> 2) * (kHalfBytes >> 4) + (kk & 3) * 2);
+        tc::mma_ss(d, dq + off, dk + off, idesc_s, kk > 0);
       }
     };
-    auto issue_pv = [&](uint32_t d, uint32_t p_tmem, uint32_t va, bool acc) {
+    auto issue_pv = [&](uint32_t d, uint32_t p_tmem, uint64_t dv, bool acc) {
 #pragma unroll
       for (int kk = 0; kk < kN / 16; ++kk)
-        tc::mma_ts(d, p_tmem + kk * 8,
-                   tc::smem_desc(va + kk * 2048, kHalfBytes, 1024, tc::kSwizzle128B), idesc_o,
-                   acc || kk > 0);
+        tc::mma_ts(d, p_tmem + kk * 8, dv + (uint64_t)(kk * (2048 >> 4)), idesc_o, acc || kk > 0);
     };
     for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
       const Unit x = unit_of(p, qoff, max_qt, u);
@@ -432,12 +438,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n; ++j, ++cnt) {
         const int s = cnt % kStages;
         const uint32_t ph = (cnt / kStages) & 1;
-        const uint32_t ka = smem_u32(smem + L::kKV + s * 2 * kTileBytes);
-        const uint32_t va = ka + kTileBytes;
+        const uint64_t dk = dk0 + (uint64_t)s * kStageStep;
+        const uint64_t dv = dv0 + (uint64_t)s * kStageStep;
         if (!(ok = wait_or_flag(bar(BAR_K_FULL + s), ph, p.dbg, abort_flag))) break;
         tc::fence_after_sync();
         if (lane == 0) {
-          issue_s(S0, q0, ka);
+          issue_s(S0, dq0, dk);
           tc::commit(bar(BAR_S_FULL + 0));
         }
         __syncwarp();
@@ -450,14 +456,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             tc::fence_after_sync();
             if (lane == 0) {
-              issue_pv(O1, S1, smem_u32(smem + L::kKV + prev_s * 2 * kTileBytes) + kTileBytes,
-                       j - 1 > 0);
+              issue_pv(O1, S1, dv0 + (uint64_t)prev_s * kStageStep, j - 1 > 0);
               tc::commit(bar(BAR_V_EMPTY + prev_s));
             }
             __syncwarp();
           }
           if (lane == 0) {
-            issue_s(S1, q1, ka);
+            issue_s(S1, dq1, dk);
             tc::commit(bar(BAR_S_FULL + 1));
           }
           __syncwarp();
@@ -481,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         tc::fence_after_sync();
         if (lane == 0) {
-          issue_pv(O0, S0, va, j > 0);
+          issue_pv(O0, S0, dv, j > 0);
           if (!p.two_heads) tc::commit(bar(BAR_V_EMPTY + s));
         }
         __syncwarp();
@@ -496,8 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         tc::fence_after_sync();
         if (lane == 0) {
-          issue_pv(O1, S1, smem_u32(smem + L::kKV + prev_s * 2 * kTileBytes) + kTileBytes,
-                   n - 1 > 0);
+          issue_pv(O1, S1, dv0 + (uint64_t)prev_s * kStageStep, n - 1 > 0);
           tc::commit(bar(BAR_V_EMPTY + prev_s));
         }
         __syncwarp();
@@ -568,13 +572,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           float mx4[4];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            float a0 = __uint_as_float(r[c][0]), a1 = __uint_as_float(r[c][1]);
+            float a0 = -INFINITY;
 #pragma unroll
-            for (int i = 2; i < 32; i += 2) {
-              a0 = fmaxf(a0, __uint_as_float(r[c][i]));
-              a1 = fmaxf(a1, __uint_as_float(r[c][i + 1]));
-            }
-            mx4[c] = fmaxf(a0, a1);
+            for (int i = 0; i < 32; i += 2)
+              a0 = fmax3(a0, __uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1]));
+            mx4[c] = a0;
           }
           mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
         }
@@ -586,31 +588,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = mxs;
         }
         const float mb = (m == -INFINITY) ? 0.f : m;
-        // pass 2, two halves of 64 columns: P = exp2(s*c - m) (masked -inf -> 0),
-        // packed in place to bf16 pairs (P[2k], P[2k+1] -> word k), stored over
-        // the first 64 columns of S
-        float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // pass 2: the row again in one round trip; P = exp2(s*c - m) (masked keys
+        // hold -inf and give 0) with the argument and the row sum on packed
+        // float pairs, packed in place to bf16 pairs (P[2k], P[2k+1] -> word k)
+        // and stored over the first 64 columns of S
+        float ls[8];
+        {
+          uint32_t r[4][32];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t r[2][32];
-          tc::ld32(S + hf * 64, r[0]);
-          tc::ld32(S + hf * 64 + 32, r[1]);
+          for (int c = 0; c < 4; ++c) tc::ld32(S + c * 32, r[c]);
           tc::wait_ld();
+          const uint64_t c2 = f2(p.scale_log2, p.scale_log2), nm2 = f2(-mb, -mb);
+          uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float e = fast_exp2(fmaf(__uint_as_float(r[c][i]), p.scale_log2, -mb));
-              ls[i & 7] += e;
-              r[c][i] = __float_as_uint(e);
-            }
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
+          for (int k = 0; k < 64; ++k) {
             const int f0 = 2 * k, f1 = 2 * k + 1;
-            r[0][k] = pack_bf16x2(__uint_as_float(r[f0 >> 5][f0 & 31]),
-                                  __uint_as_float(r[f1 >> 5][f1 & 31]));
+            const uint64_t xv = ffma2(
+                f2(__uint_as_float(r[f0 >> 5][f0 & 31]), __uint_as_float(r[f1 >> 5][f1 & 31])),
+                c2, nm2);
+            float x0, x1;
+            f2_split(xv, x0, x1);
+            const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+            acc[k & 3] = fadd2(acc[k & 3], f2(e0, e1));
+            r[k >> 5][k & 31] = pack_bf16x2(e0, e1);
           }
-          tc::st32(S + hf * 32, r[0]);
+          tc::st32(S, r[0]);
+          tc::st32(S + 32, r[1]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) f2_split(acc[k], ls[2 * k], ls[2 * k + 1]);
         }
         const float ls0 = (ls[0] + ls[1]) + (ls[2] + ls[3]);
         const float ls1 = (ls[4] + ls[5]) + (ls[6] + ls[7]);
