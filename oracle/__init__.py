@@ -41,4 +41,5 @@ from .attention64 import (  # noqa: F401
     paged_decode_rows,
     kv_append,
     kv_gather,
+    kv_copy_blocks,
 )

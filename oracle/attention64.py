@@ -292,3 +292,15 @@ def kv_gather(k_cache, v_cache, block_tables, seq_lens, out_max_len):
         vo[b, :, :L, :] = v_cache[blocks, :, rows, :].transpose(1, 0, 2) \
             if not hasattr(v_cache, "detach") else v_cache[blocks, :, rows, :].transpose(0, 1)
     return ko, vo
+
+
+def kv_copy_blocks(k_cache, v_cache, block_pairs):
+    """Expected pools after copy-on-write: for each (src, dst) pair, block dst
+    becomes a copy of block src (all KV heads, K and V). Copies, inputs are not
+    modified; destinations are assumed distinct and not sources."""
+    kc = k_cache.clone() if hasattr(k_cache, "clone") else np.array(k_cache, copy=True)
+    vc = v_cache.clone() if hasattr(v_cache, "clone") else np.array(v_cache, copy=True)
+    for src, dst in _i64(block_pairs).reshape(-1, 2):
+        kc[dst] = k_cache[src]
+        vc[dst] = v_cache[src]
+    return kc, vc

@@ -409,3 +409,13 @@ def test_gather_brute_force():
                     assert torch.equal(vo[b, h, p], vc[tab[b, p // 4], h, p % 4])
                 else:
                     assert torch.all(ko[b, h, p] == 0) and torch.all(vo[b, h, p] == 0)
+
+
+def test_copy_blocks_brute_force():
+    kc = torch.arange(6 * 2 * 4 * 3, dtype=torch.float32).view(6, 2, 4, 3)
+    vc = -kc
+    ek, ev = oracle.kv_copy_blocks(kc, vc, [[1, 4], [5, 0]])
+    for blk in range(6):
+        src = {4: 1, 0: 5}.get(blk, blk)
+        assert torch.equal(ek[blk], kc[src]) and torch.equal(ev[blk], vc[src])
+    assert torch.equal(kc, torch.arange(6 * 2 * 4 * 3, dtype=torch.float32).view(6, 2, 4, 3))
