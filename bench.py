@@ -58,12 +58,12 @@ def peaks():
 # after any change to them the bench reports null until they are profiled again.
 PROFILED_TRAFFIC = {
     "decode": {"sources": ['csrc/decode.cu', 'csrc/pkv_common.cuh'],
-               "sha256": "f1968cf1c3212cc986b1c73324cfd7316f253afe4c997a4d72fd254c89b61551",
-               "per_unit": 194937344 / 190134992,  # per algorithmic byte (16-seq ragged case)
+               "sha256": "4c37c4b9b05470cef1de74ba2b67369535fbe198e78a6f0b2b0c27b9c0491288",
+               "per_unit": 194804224 / 190134992,  # per algorithmic byte (16-seq ragged case)
                },
     "prefill": {"sources": ['csrc/prefill.cu', 'csrc/pkv_common.cuh', 'csrc/tc_sm100.cuh'],
-                "sha256": "4dc33d68e9819d7d3630fa72963d01a2e87df90a997ea37017c996f5990e4372",
-                "per_unit": 299044608 / 1065168666624,  # per causal FLOP (1-seq case)
+                "sha256": "c512983f32c3b9e728518ba3b9d0fe44f058ca87beeaf776300f53053a4e4b78",
+                "per_unit": 298265088 / 1065168666624,  # per causal FLOP (1-seq case)
                 },
 }
 

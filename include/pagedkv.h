@@ -128,6 +128,20 @@ PKV_API int paged_kv_gather(const void* k_cache, const void* v_cache, pkv_cache_
                     void* v_out, int32_t* dbg_err, void* stream);
 
 /*
+ * paged_kv_copy_blocks — copy-on-write of shared blocks.
+ * Source: "Ultimate Guide to PagedAttention", memory-sharing section: shared
+ * blocks are stored once and copied when one of their holders writes to them.
+ *   block_pairs  int32 [num_pairs, 2] device: (src, dst) physical block ids.
+ * Every KV head's rows of block src are copied to block dst, in K and in V,
+ * exactly. A dst must not appear twice nor be a src of another pair in the
+ * same call (the copies run concurrently). Ids outside [0, num_blocks) skip
+ * the pair and set PKV_DBG_BLOCK_ID.
+ */
+PKV_API int paged_kv_copy_blocks(void* k_cache, void* v_cache, pkv_cache_desc cache,
+                                 const int32_t* block_pairs, int32_t num_pairs,
+                                 int32_t* dbg_err, void* stream);
+
+/*
  * paged_attention_decode_workspace_size — bytes of scratch the decode call
  * needs on the current device (depends on the device's SM count, the group
  * size num_q_heads/num_kv_heads, head_dim and batch). 0 for float32 pools.

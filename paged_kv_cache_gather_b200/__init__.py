@@ -4,6 +4,7 @@ Calls (thin bindings over the C ABI in ``include/pagedkv.h``):
 
 * ``paged_kv_append``         slot-mapped write of new tokens' K/V
 * ``paged_kv_gather``         block tables resolved to contiguous K/V
+* ``paged_kv_copy_blocks``    copy-on-write of shared blocks
 * ``paged_attention_decode``  one query per sequence over paged KV
 * ``paged_attention_prefill`` a chunk of queries over paged context + chunk
 
@@ -21,6 +22,7 @@ from .ops import (  # noqa: F401
     paged_attention_decode,
     paged_attention_prefill,
     paged_kv_append,
+    paged_kv_copy_blocks,
     paged_kv_gather,
     read_dbg,
     sliding_window,

@@ -35,6 +35,7 @@ PKV_MASK_SLIDING = 2
 EXPORTS = (
     "paged_kv_append",
     "paged_kv_gather",
+    "paged_kv_copy_blocks",
     "paged_attention_decode_workspace_size",
     "paged_attention_decode",
     "paged_attention_prefill",
@@ -78,6 +79,8 @@ def _declare(lib):
     lib.paged_kv_gather.argtypes = [_vp, _vp, CacheDescC, _vp, _i32, _vp, _i32, _i32, _vp, _vp,
                                     _vp, _vp]
     lib.paged_kv_gather.restype = ctypes.c_int
+    lib.paged_kv_copy_blocks.argtypes = [_vp, _vp, CacheDescC, _vp, _i32, _vp, _vp]
+    lib.paged_kv_copy_blocks.restype = ctypes.c_int
     lib.paged_attention_decode_workspace_size.argtypes = [_i32, _i32, CacheDescC]
     lib.paged_attention_decode_workspace_size.restype = _sz
     lib.paged_attention_decode.argtypes = [_vp, _vp, _vp, CacheDescC, _vp, _i32, _vp, _i32, _i32,

@@ -169,6 +169,21 @@ int paged_kv_gather(const void* k_cache, const void* v_cache, pkv_cache_desc cac
                        out_max_len, k_out, v_out, dbg_err, static_cast<cudaStream_t>(stream));
 }
 
+int paged_kv_copy_blocks(void* k_cache, void* v_cache, pkv_cache_desc cache,
+                         const int32_t* block_pairs, int32_t num_pairs, int32_t* dbg_err,
+                         void* stream) {
+  g_last_error[0] = 0;
+  if (int st = check_cache(cache, "paged_kv_copy_blocks")) return st;
+  if (num_pairs < 0) return fail(PKV_ERR_INVALID_ARG, "paged_kv_copy_blocks: num_pairs < 0");
+  if (num_pairs == 0) return PKV_OK;
+  if (!k_cache || !v_cache || !block_pairs)
+    return fail(PKV_ERR_INVALID_ARG, "paged_kv_copy_blocks: null pointer");
+  if (!aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PKV_ERR_INVALID_ARG, "paged_kv_copy_blocks: pools must be 16-byte aligned");
+  return launch_copy_blocks(k_cache, v_cache, cache, block_pairs, num_pairs, dbg_err,
+                            static_cast<cudaStream_t>(stream));
+}
+
 size_t paged_attention_decode_workspace_size(int32_t batch, int32_t num_q_heads,
                                              pkv_cache_desc cache) {
   if (check_cache(cache, "paged_attention_decode_workspace_size") != PKV_OK) return 0;

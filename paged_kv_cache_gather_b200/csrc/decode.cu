@@ -721,7 +721,17 @@ int launch_bf16_impl(const DecodeArgs& a) {
   decode_bf16_kernel<D, NSTAGE, WPC><<<sms, WPC * 32, smem, a.stream>>>(kmap, vmap, p);
   if (int st = check_launch("paged_attention_decode")) return st;
   const int64_t items = (int64_t)a.batch * a.cache.num_kv_heads * g;
-  decode_combine_kernel<D><<<(unsigned)((items + 3) / 4), 128, 0, a.stream>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((items + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = a.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, p);
   return check_launch("paged_attention_decode: combine");
 }
 

@@ -127,6 +127,21 @@ def paged_kv_gather(k_cache, v_cache, block_tables, seq_lens, out_max_len, dbg_e
     return ko, vo
 
 
+def paged_kv_copy_blocks(k_cache, v_cache, block_pairs, dbg_err=None):
+    """Copy-on-write: copy every KV head of block src to block dst for each
+    (src, dst) row of ``block_pairs`` (int32 [n, 2] on the device)."""
+    _check_pool(k_cache, v_cache)
+    dev = k_cache.device
+    if isinstance(block_pairs, (list, tuple)):
+        block_pairs = torch.tensor(block_pairs, dtype=torch.int32, device=dev).view(-1, 2)
+    _check(block_pairs.dtype == torch.int32 and block_pairs.device == dev and
+           block_pairs.is_contiguous() and block_pairs.dim() == 2 and block_pairs.shape[1] == 2,
+           "block_pairs must be a contiguous int32 [n, 2] tensor on the device")
+    L.check(L.lib().paged_kv_copy_blocks(_ptr(k_cache), _ptr(v_cache), cache_desc(k_cache),
+                                         _ptr(block_pairs), block_pairs.shape[0], _ptr(dbg_err),
+                                         _stream()))
+
+
 def decode_workspace_size(batch, num_q_heads, k_cache):
     return int(L.lib().paged_attention_decode_workspace_size(batch, num_q_heads,
                                                              cache_desc(k_cache)))
