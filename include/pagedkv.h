@@ -205,6 +205,50 @@ PKV_API int paged_attention_prefill(const void* q, const void* k_new, const void
                             void* out, float* lse, int32_t* dbg_err, void* stream);
 
 /*
+ * paged_attention_decode_shared_prefix_workspace_size — bytes of scratch the
+ * shared-prefix decode call needs (the decode workspace plus float32
+ * partials for every (sequence, query head)). 0 on invalid arguments.
+ */
+PKV_API size_t paged_attention_decode_shared_prefix_workspace_size(int32_t batch,
+                                                                   int32_t num_q_heads,
+                                                                   pkv_cache_desc cache);
+
+/*
+ * paged_attention_decode_shared_prefix — paged_attention_decode for batches
+ * whose sequences come in groups (beams, parallel samples) that share a
+ * prompt stored once. Source: "Ultimate Guide to PagedAttention", memory
+ * sharing and beam search (sequences of one request map their common
+ * prefix to the same physical blocks); the result is exact, the softmax over
+ * prefix and private keys being the log-sum-exp merge of the two parts
+ * ("FlashAttention", exact tiled attention). Each shared block is read once
+ * per group and KV head instead of once per sequence.
+ * Same arguments, layouts, results and errors as paged_attention_decode, plus:
+ *   group_start     int32 [num_groups + 1] on the device: group i holds batch
+ *                   entries group_start[i] .. group_start[i+1]-1; groups tile
+ *                   0 .. batch-1 in order (group_start[0] = 0, last = batch).
+ *   max_group_size  host int, >= every group's size; max_group_size *
+ *                   (num_q_heads / num_kv_heads) must be <= 128.
+ *   shared_len      int32 [batch] on the device: keys 0 .. shared_len[b]-1
+ *                   of sequence b are the group's shared prefix. All members
+ *                   of a group give the same value, 0 <= shared_len[b] <=
+ *                   seq_lens[b], and those keys must hold the same K/V in
+ *                   every member (normally the same physical blocks; the
+ *                   call reads them through the group's first member's table).
+ *   workspace       >= paged_attention_decode_shared_prefix_workspace_size().
+ * A group whose shared length is 0 reduces to plain decode for its members.
+ * Violations of the group rules are flagged in dbg_err (PKV_DBG_LENGTH).
+ * Supported: BF16, head_dim 128, block_size >= 8, masks none and causal
+ * (a decode query sees its whole context under both).
+ */
+PKV_API int paged_attention_decode_shared_prefix(
+    const void* q, const void* k_cache, const void* v_cache, pkv_cache_desc cache,
+    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+    int32_t batch, int32_t num_q_heads, float scale, pkv_mask_mod mask,
+    const int32_t* group_start, int32_t num_groups, int32_t max_group_size,
+    const int32_t* shared_len, void* out, float* lse, void* workspace, size_t workspace_bytes,
+    int32_t* dbg_err, void* stream);
+
+/*
  * paged_attention_decode_noalloc — paged_attention_decode without a
  * caller-provided workspace. The pages have no counterpart to this call: it
  * exists for callers that cannot allocate device memory (a runtime whose

@@ -7,6 +7,8 @@ Calls (thin bindings over the C ABI in ``include/pagedkv.h``):
 * ``paged_kv_copy_blocks``    copy-on-write of shared blocks
 * ``paged_attention_decode``  one query per sequence over paged KV
 * ``paged_attention_prefill`` a chunk of queries over paged context + chunk
+* ``paged_attention_decode_shared_prefix``  decode for groups (beams,
+  samples) sharing a prefix, each shared block read once per group
 
 Host helpers: ``BlockManager`` (free list, tables, refcounts, copy-on-write)
 and the seeded workload generators in ``inputs``.
@@ -20,11 +22,14 @@ from .ops import (  # noqa: F401
     decode_workspace_size,
     no_mask,
     paged_attention_decode,
+    paged_attention_decode_shared_prefix,
     paged_attention_prefill,
     paged_kv_append,
     paged_kv_copy_blocks,
     paged_kv_gather,
     read_dbg,
+    shared_prefix_workspace,
+    shared_prefix_workspace_size,
     sliding_window,
 )
 from ._lib import PagedKVError  # noqa: F401

@@ -40,6 +40,8 @@ EXPORTS = (
     "paged_attention_decode",
     "paged_attention_prefill",
     "paged_attention_decode_noalloc",
+    "paged_attention_decode_shared_prefix_workspace_size",
+    "paged_attention_decode_shared_prefix",
     "pkv_debug_exp2",
     "pkv_status_string",
     "pkv_last_error",
@@ -93,6 +95,12 @@ def _declare(lib):
     lib.paged_attention_decode_noalloc.argtypes = [_vp, _vp, _vp, CacheDescC, _vp, _i32, _vp, _i32,
                                                    _i32, _f32, MaskModC, _vp, _vp, _vp, _vp]
     lib.paged_attention_decode_noalloc.restype = ctypes.c_int
+    lib.paged_attention_decode_shared_prefix_workspace_size.argtypes = [_i32, _i32, CacheDescC]
+    lib.paged_attention_decode_shared_prefix_workspace_size.restype = _sz
+    lib.paged_attention_decode_shared_prefix.argtypes = [
+        _vp, _vp, _vp, CacheDescC, _vp, _i32, _vp, _i32, _i32, _f32, MaskModC, _vp, _i32, _i32,
+        _vp, _vp, _vp, _vp, _sz, _vp, _vp]
+    lib.paged_attention_decode_shared_prefix.restype = ctypes.c_int
     lib.pkv_debug_exp2.argtypes = [_vp, _vp, _i32, _vp]
     lib.pkv_debug_exp2.restype = ctypes.c_int
     lib.pkv_status_string.argtypes = [ctypes.c_int]

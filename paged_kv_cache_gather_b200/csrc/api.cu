@@ -23,6 +23,8 @@ int fail(int status, const char* fmt, ...) {
   return status;
 }
 
+void clear_last_error() { g_last_error[0] = 0; }
+
 int device_sm_count() {
   static int cached[64] = {0};
   int dev = 0;
@@ -90,9 +92,7 @@ bool make_tensor_map_bf16(void* map_out, const void* base, int rank, const uint6
   return r == CUDA_SUCCESS;
 }
 
-static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
-
-static int check_cache(const pkv_cache_desc& c, const char* fn) {
+int check_cache(const pkv_cache_desc& c, const char* fn) {
   if (c.num_blocks <= 0 || c.num_kv_heads <= 0 || c.head_dim <= 0 || c.block_size <= 0)
     return fail(PKV_ERR_INVALID_ARG, "%s: cache sizes must be positive", fn);
   if (c.block_size & (c.block_size - 1))
@@ -109,7 +109,7 @@ static int check_cache(const pkv_cache_desc& c, const char* fn) {
   return PKV_OK;
 }
 
-static int check_mask(const pkv_mask_mod& m, const char* fn) {
+int check_mask(const pkv_mask_mod& m, const char* fn) {
   if (m.kind != PKV_MASK_NONE && m.kind != PKV_MASK_CAUSAL && m.kind != PKV_MASK_SLIDING)
     return fail(PKV_ERR_INVALID_ARG, "%s: unknown mask kind %d", fn, m.kind);
   return PKV_OK;

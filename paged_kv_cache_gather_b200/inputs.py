@@ -270,8 +270,89 @@ def config4(groups=8, beams=8, prefix=4096, suffix=256, num_blocks=4096, shared=
                      Hkv, Hq, d, k_cache, v_cache, tables, seq_lens, 1.0 / float(np.sqrt(d)),
                      MASK_CAUSAL, 0, None, q)
     case.extra["unique_blocks"] = len(set(int(x) for r in rows for x in r))
+    case.extra["group_start"] = torch.arange(0, B + 1, beams, dtype=torch.int32)
+    case.extra["shared_len"] = torch.full((B,), prefix if shared else 0, dtype=torch.int32)
+    case.extra["max_group_size"] = beams
     if peaky:
         make_peaky(case, s + 7)
+    return case
+
+
+def make_shared_prefix_case(name, *, group_sizes, prefix_lens, suffix_lens, num_q_heads=32,
+                            num_kv_heads=8, head_dim=128, block_size=16, spare_blocks=64,
+                            seed, mask_kind=MASK_CAUSAL, peaky=False):
+    """Groups of decode sequences that share a prefix, laid out as a fork leaves them.
+
+    Group ``i`` has ``group_sizes[i]`` members and a prefix of
+    ``prefix_lens[i]`` tokens; member ``b`` then has ``suffix_lens[b]`` tokens
+    of its own. The prefix's full blocks are one set of block ids in every
+    member's table. When the prefix ends inside a block, every member holds its
+    own copy of that block (as after a copy-on-write): the prefix rows are the
+    first member's values, the rows after them the member's own. Tables come
+    from one seeded permutation of the pool; the query of each sequence sits at
+    its last position. ``extra`` gets ``group_start`` (int32 [G+1]),
+    ``shared_len`` (int32 [B]), ``max_group_size`` and ``unique_blocks``.
+    """
+    gen = torch.Generator().manual_seed(seed)
+    rng = np.random.default_rng(seed)
+    bs = block_size
+    group_sizes = [int(n) for n in group_sizes]
+    B = sum(group_sizes)
+    if len(prefix_lens) != len(group_sizes) or len(suffix_lens) != B:
+        raise ValueError("prefix_lens needs one entry per group, suffix_lens one per sequence")
+    need, b = 0, 0
+    for gi, n in enumerate(group_sizes):
+        need += prefix_lens[gi] // bs
+        for _ in range(n):
+            L = prefix_lens[gi] + suffix_lens[b]
+            need += (L + bs - 1) // bs - prefix_lens[gi] // bs
+            b += 1
+    pool = need + spare_blocks
+    free = rng.permutation(pool)
+    k_cache = randn((pool, num_kv_heads, bs, head_dim), gen)
+    v_cache = randn((pool, num_kv_heads, bs, head_dim), gen)
+    rows, lens, shared, starts, partial = [], [], [], [0], []
+    pos, b = 0, 0
+    for gi, n in enumerate(group_sizes):
+        P = int(prefix_lens[gi])
+        full = P // bs
+        pre = free[pos:pos + full].tolist()
+        pos += full
+        leader_row = None
+        for _ in range(n):
+            L = P + int(suffix_lens[b])
+            own = (L + bs - 1) // bs - full
+            r = pre + free[pos:pos + own].tolist()
+            pos += own
+            rows.append(r)
+            lens.append(L)
+            shared.append(P)
+            if leader_row is None:
+                leader_row = r
+            elif P % bs and own > 0:
+                partial.append((leader_row[full], r[full], P % bs))
+            b += 1
+        starts.append(starts[-1] + n)
+    width = max(1, max(len(r) for r in rows))
+    tables = _table_tensor(rows, width)
+    seq_lens = torch.tensor(lens, dtype=torch.int32)
+    q = randn((B, num_q_heads, head_dim), gen)
+    case = PagedCase(name, torch.bfloat16, pool, bs, num_kv_heads, num_q_heads, head_dim, k_cache,
+                     v_cache, tables, seq_lens, 1.0 / float(np.sqrt(head_dim)), mask_kind, 0,
+                     None, q)
+    if peaky:
+        make_peaky(case, seed + 7)
+
+    def copy_prefix_rows():
+        for src, dst, r in partial:
+            case.k_cache[dst, :, :r] = case.k_cache[src, :, :r]
+            case.v_cache[dst, :, :r] = case.v_cache[src, :, :r]
+
+    copy_prefix_rows()
+    case.extra["group_start"] = torch.tensor(starts, dtype=torch.int32)
+    case.extra["shared_len"] = torch.tensor(shared, dtype=torch.int32)
+    case.extra["max_group_size"] = max(group_sizes)
+    case.extra["unique_blocks"] = len(set(int(x) for r in rows for x in r))
     return case
 
 

@@ -182,6 +182,57 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, seq_lens, scale=No
     return out, lse
 
 
+def shared_prefix_workspace_size(batch, num_q_heads, k_cache):
+    return int(L.lib().paged_attention_decode_shared_prefix_workspace_size(
+        batch, num_q_heads, cache_desc(k_cache)))
+
+
+def shared_prefix_workspace(batch, num_q_heads, k_cache):
+    n = shared_prefix_workspace_size(batch, num_q_heads, k_cache)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=k_cache.device)
+
+
+def paged_attention_decode_shared_prefix(q, k_cache, v_cache, block_tables, seq_lens,
+                                         group_start, shared_len, max_group_size, scale=None,
+                                         mask_mod: Optional[MaskMod] = None, *, out=None,
+                                         lse=None, workspace=None, dbg_err=None):
+    """Decode for groups of sequences (beams, samples) that share a prefix.
+
+    ``group_start`` (int32 [G+1] on the device) splits the batch into
+    consecutive groups; ``shared_len`` (int32 [B]) is the length of each
+    sequence's shared prefix, the same within a group. ``max_group_size`` is a
+    host int bounding every group's size. Returns (out, lse) equal to
+    ``paged_attention_decode`` on the same inputs."""
+    _check_pool(k_cache, v_cache)
+    dev = k_cache.device
+    _i32(block_tables, "block_tables", dev)
+    _i32(seq_lens, "seq_lens", dev)
+    _i32(group_start, "group_start", dev)
+    _i32(shared_len, "shared_len", dev)
+    B, Hq, d = q.shape
+    _check(q.dtype == k_cache.dtype and q.device == dev and q.is_contiguous(),
+           "q must be contiguous, on the cache's device, in the cache dtype")
+    _check(d == k_cache.shape[3], "head_dim mismatch")
+    _check(block_tables.dim() == 2 and block_tables.shape[0] == B and seq_lens.numel() == B
+           and shared_len.numel() == B, "block_tables, seq_lens and shared_len must match q")
+    _check(group_start.dim() == 1 and group_start.numel() >= 2, "group_start must be [G + 1]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    mask_mod = mask_mod or no_mask()
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = shared_prefix_workspace(B, Hq, k_cache)
+    L.check(L.lib().paged_attention_decode_shared_prefix(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), cache_desc(k_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(seq_lens), B, Hq, float(scale), mask_mod.to_c(B, dev),
+        _ptr(group_start), group_start.numel() - 1, int(max_group_size), _ptr(shared_len),
+        _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _ptr(dbg_err), _stream()))
+    return out, lse
+
+
 def paged_attention_prefill(q, k_new, v_new, k_cache, v_cache, block_tables, ctx_lens, q_lens,
                             mask_mod: Optional[MaskMod] = None, scale=None, *, out=None,
                             lse=None, dbg_err=None):
