@@ -355,8 +355,9 @@ def decode_sweep(dev, flush):
 
 def shared_prefix(dev, flush):
     """8 groups x 8 beams, 4096-token prefix shared by block id + 256 own tokens:
-    decode time with shared blocks and with copied ones; logical bytes are what
-    the beams read, unique bytes what is stored."""
+    plain decode time with shared blocks and with copied ones, and the grouped
+    (shared-prefix) call on the shared layout; logical bytes are what the beams
+    attend over, unique bytes what is stored."""
     import paged_kv_cache_gather_b200 as pkv
     from paged_kv_cache_gather_b200 import inputs as I
 
@@ -378,8 +379,25 @@ def shared_prefix(dev, flush):
         out["shared" if shared else "copied"] = {
             "us": round(ms * 1e3, 2), "logical_GBps": round(logical / (ms * 1e-3) / 1e9, 1),
             "unique_bytes": unique, "unique_GBps": round(unique / (ms * 1e-3) / 1e9, 1)}
+        if shared:
+            # the grouped call: prefix once per (group, KV head), own keys, merge
+            gs = c.extra["group_start"].to(dev)
+            sl = c.extra["shared_len"].to(dev)
+            wsg = pkv.shared_prefix_workspace(q.shape[0], q.shape[1], kc)
+            grouped = lambda: pkv.paged_attention_decode_shared_prefix(
+                q, kc, vc, tab, lens, gs, sl, c.extra["max_group_size"], c.scale, pkv.causal(),
+                out=o, lse=lse, workspace=wsg)
+            for _ in range(3):
+                grouped()
+            ms_g = time_calls(grouped, 20, flush)
+            out["grouped"] = {
+                "us": round(ms_g * 1e3, 2),
+                "logical_GBps": round(logical / (ms_g * 1e-3) / 1e9, 1),
+                "unique_GBps": round(unique / (ms_g * 1e-3) / 1e9, 1),
+                "launches": 2}
         del kc, vc
         torch.cuda.empty_cache()
+    out["grouped_speedup_vs_shared"] = round(out["shared"]["us"] / out["grouped"]["us"], 2)
     return out
 
 

@@ -206,8 +206,10 @@ PKV_API int paged_attention_prefill(const void* q, const void* k_new, const void
 
 /*
  * paged_attention_decode_shared_prefix_workspace_size — bytes of scratch the
- * shared-prefix decode call needs (the decode workspace plus float32
- * partials for every (sequence, query head)). 0 on invalid arguments.
+ * shared-prefix decode call needs on the current device (float32 pieces of
+ * split segments for every worker, per-(sequence, head) results of the prefix
+ * and of the own keys, a tile prefix over the work items). 0 on invalid
+ * arguments.
  */
 PKV_API size_t paged_attention_decode_shared_prefix_workspace_size(int32_t batch,
                                                                    int32_t num_q_heads,
@@ -218,27 +220,33 @@ PKV_API size_t paged_attention_decode_shared_prefix_workspace_size(int32_t batch
  * whose sequences come in groups (beams, parallel samples) that share a
  * prompt stored once. Source: "Ultimate Guide to PagedAttention", memory
  * sharing and beam search (sequences of one request map their common
- * prefix to the same physical blocks); the result is exact, the softmax over
- * prefix and private keys being the log-sum-exp merge of the two parts
- * ("FlashAttention", exact tiled attention). Each shared block is read once
- * per group and KV head instead of once per sequence.
+ * prefix to the same physical blocks). Each sequence's attention is split
+ * into its group's shared prefix and its own keys and the two parts are
+ * merged by log-sum-exp, which is exact ("FlashAttention", exact tiled
+ * attention). The prefix is attended once per group and KV head with every
+ * member's query heads together, so each shared block is read once per group
+ * instead of once per sequence. Two kernel launches on `stream`.
  * Same arguments, layouts, results and errors as paged_attention_decode, plus:
  *   group_start     int32 [num_groups + 1] on the device: group i holds batch
  *                   entries group_start[i] .. group_start[i+1]-1; groups tile
  *                   0 .. batch-1 in order (group_start[0] = 0, last = batch).
+ *   num_groups      host int, 1 .. batch.
  *   max_group_size  host int, >= every group's size; max_group_size *
  *                   (num_q_heads / num_kv_heads) must be <= 128.
  *   shared_len      int32 [batch] on the device: keys 0 .. shared_len[b]-1
- *                   of sequence b are the group's shared prefix. All members
+ *                   of sequence b are its group's shared prefix. All members
  *                   of a group give the same value, 0 <= shared_len[b] <=
- *                   seq_lens[b], and those keys must hold the same K/V in
- *                   every member (normally the same physical blocks; the
- *                   call reads them through the group's first member's table).
- *   workspace       >= paged_attention_decode_shared_prefix_workspace_size().
+ *                   seq_lens[b], and those keys hold the same K/V in every
+ *                   member (normally the same physical blocks; the call reads
+ *                   them through the first member's block table).
+ *   workspace       >= paged_attention_decode_shared_prefix_workspace_size()
+ *                   bytes, 16-byte aligned; calls sharing it must not overlap.
  * A group whose shared length is 0 reduces to plain decode for its members.
- * Violations of the group rules are flagged in dbg_err (PKV_DBG_LENGTH).
- * Supported: BF16, head_dim 128, block_size >= 8, masks none and causal
- * (a decode query sees its whole context under both).
+ * Group descriptions that break these rules are flagged in dbg_err
+ * (PKV_DBG_LENGTH); the affected rows then skip the prefix.
+ * Supported: BF16, head_dim 128, block_size >= 8, at most 32 query heads per
+ * KV head, masks none and causal (a decode query sees its whole context
+ * under both).
  */
 PKV_API int paged_attention_decode_shared_prefix(
     const void* q, const void* k_cache, const void* v_cache, pkv_cache_desc cache,

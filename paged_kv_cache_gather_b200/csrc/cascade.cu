@@ -1,23 +1,38 @@
-// Shared-prefix (cascade) decode: beams or samples that share a prompt read
-// its KV blocks once per group instead of once per sequence.
+// Shared-prefix (cascade) decode: sequences that share a prompt (beams,
+// parallel samples) read its KV blocks once per group instead of once each.
 //
 // Source: "Ultimate Guide to PagedAttention", sections on memory sharing and
-// beam search (requests with a common prefix point at the same physical
-// blocks, stored once); the split into a shared part and a private part is
-// exact because softmax attention over a union of key sets is the
-// log-sum-exp merge of the attention over each part ("FlashAttention",
-// abstract: exact attention computed tile by tile).
+// beam search (sequences of one request point their common prefix at the same
+// physical blocks, stored once). Splitting each sequence's keys into the
+// shared prefix and its own keys is exact: softmax attention over a union of
+// key sets is the log-sum-exp merge of the attention over each set, the same
+// identity the tiled exact softmax of "FlashAttention" (abstract) rests on.
 //
-// Three launches on the caller's stream:
-//  1. prefix: the tensor-core prefill kernel in group mode; a unit is (group,
-//     KV head) with every member's query heads as the rows of one query tile
-//     (8 beams x 4 heads = 32 rows), so each shared block is loaded once per
-//     group and KV head; float32 partials (o, lse) per (sequence, head);
-//  2. suffix: the regular paged decode over each sequence's keys from its
-//     shared length on (per-sequence key start), written to out and to an
-//     internal lse;
-//  3. merge: o = w_p o_p + w_s o_s with w = exp(lse_part - lse),
-//     lse = log(exp(lse_p) + exp(lse_s)), in place over out.
+// B200 design (bf16, head_dim 128):
+//  * One persistent launch of `grouped_decode_kernel` over a flat list of
+//    16-token tiles, as in the paged decode kernel. An item of the list is
+//    either a prefix item (one group, up to 32 query rows: every member's
+//    query heads of a KV head, row = member * g + head; keys: the group's
+//    shared prefix through its first member's block table) or an own-key item
+//    (one sequence, its g query heads; keys from its shared length to its
+//    end). Each (item, KV head) segment is a run of tiles; warps take equal
+//    contiguous ranges of the whole list, so the work is balanced whatever the
+//    group sizes and lengths are.
+//  * The query rows of a segment are the N side of mma.sync m16n8k16 (four
+//    n-tiles of 8 rows), so a KV tile, loaded once by TMA into the warp's ring,
+//    serves all members of the group. S^T = K Q^T puts tokens on M; P^T is
+//    transposed in registers (movmatrix) into the B operand of O^T += V^T P^T.
+//    The query tile of a segment is staged in the warp's shared memory
+//    (128-byte XOR swizzle) and read with ldmatrix. The path is HBM-bound: a
+//    tile of 8 KB carries up to 64 small MMAs.
+//  * Results leave the main kernel normalised, in float32: a segment one warp
+//    did whole goes to a per-(sequence, head) buffer (one for prefixes, one for
+//    own keys); a segment cut between warps leaves pieces in per-warp slots.
+//    `grouped_combine_kernel` (a programmatic dependent launch) gives each
+//    (sequence, head) one warp that finds the sequence's group, merges the
+//    pieces of its prefix segment and of its own-key segment by log-sum-exp,
+//    merges the two, and writes bf16 out and the LSE.
+#include <climits>
 #include <cmath>
 
 #include "pkv_common.cuh"
@@ -28,51 +43,660 @@ namespace pkv {
 namespace {
 
 constexpr int kD = 128;
+constexpr int kTile = 16;            // tokens per tile
+constexpr int kRows = 32;            // query rows per segment (4 n-tiles of 8)
+constexpr int kNT = kRows / 8;
+constexpr int kWarps = 8;            // warps per CTA, one CTA per SM
+constexpr int kStages = 2;           // TMA ring depth per warp
+constexpr int kMinTilesPerWorker = 2;
+constexpr int kTileBytes = kTile * kD * 2;            // K (or V) bytes of one tile
+constexpr int kStageBytes = 2 * kTileBytes;           // K then V
+constexpr int kQBytes = kRows * kD * 2;               // staged query rows of a segment
+constexpr int kWarpSmem = kStages * kStageBytes + kQBytes;
 
-__global__ void __launch_bounds__(128) shared_prefix_merge_kernel(
-    __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out, const float* __restrict__ part_o,
-    const float* __restrict__ part_lse, const float* __restrict__ lse_s,
-    const int32_t* __restrict__ shared_len, int32_t batch, int32_t num_q_heads) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);  // (sequence, head)
-  if (row >= (int64_t)batch * num_q_heads) return;
-  const int b = (int)(row / num_q_heads);
-  const float ls = lse_s[row];
-  float lse = ls;
-  if (shared_len[b] > 0) {
-    const float lp = part_lse[row];
-    const float m = fmaxf(lp, ls);
-    if (m != -INFINITY) {
-      const float wp = expf(lp - m), ws = expf(ls - m);
-      const float inv = 1.f / (wp + ws);
-      lse = m + logf(wp + ws);
-      const float4 po = reinterpret_cast<const float4*>(part_o + row * kD)[lane];
-      uint2 sv = reinterpret_cast<const uint2*>(out + row * kD)[lane];
-      const float s0 = __uint_as_float(sv.x << 16), s1 = __uint_as_float(sv.x & 0xffff0000u);
-      const float s2 = __uint_as_float(sv.y << 16), s3 = __uint_as_float(sv.y & 0xffff0000u);
-      const float a = wp * inv, c = ws * inv;
-      uint2 r;
-      r.x = pack_bf16x2(a * po.x + c * s0, a * po.y + c * s1);
-      r.y = pack_bf16x2(a * po.z + c * s2, a * po.w + c * s3);
-      reinterpret_cast<uint2*>(out + row * kD)[lane] = r;
-    }
-  }
-  if (lse_out && lane == 0) lse_out[row] = lse;
-}
-
-struct Layout {
-  size_t dec, part_o, part_lse, lse_s, total;
+struct GroupedParams {
+  const __nv_bfloat16* q;      // [batch, Hq, D]
+  const int32_t* tables;
+  int32_t max_blocks;
+  const int32_t* seq_lens;
+  const int32_t* group_start;  // [num_groups + 1]
+  const int32_t* shared_len;   // [batch]
+  int32_t batch;
+  int32_t num_groups;
+  int32_t row_blocks;          // prefix items per group: ceil(max_members * g / kRows)
+  int32_t max_members;
+  int32_t items;               // num_groups * row_blocks + batch
+  int32_t num_kv_heads;
+  int32_t group;               // query heads per KV head
+  int32_t num_q_heads;
+  int32_t bs_shift;
+  int32_t num_blocks;
+  float scale_log2;
+  __nv_bfloat16* out;
+  float* lse;
+  float* ws_o;                 // [2 * workers, kRows, D] pieces of split segments
+  float* ws_lse;               // [2 * workers, kRows]
+  float* whole_o;              // [2, batch * Hq, D]: prefix (0) / own keys (1), whole segments
+  float* whole_lse;            // [2, batch * Hq]
+  int32_t* ws_prefix;          // [items + 1] tiles per KV head before item i
+  int32_t workers;
+  int32_t* dbg;
 };
 
-Layout layout(int32_t batch, int32_t num_q_heads, const pkv_cache_desc& c) {
+// One entry of the work list.
+struct Item {
+  int lo, hi;    // keys [lo, hi)
+  int t0, n;     // first tile (16-token units of position) and number of tiles
+  int lead;      // sequence whose block table holds the keys (and first query row)
+  int rows;      // query rows of the segment
+  int rb;        // row block within the group (prefix items)
+  bool prefix;
+};
+
+__device__ __forceinline__ int clamp_len(const GroupedParams& p, int L) {
+  const int cap = p.max_blocks << p.bs_shift;
+  if (L > cap) {
+    flag_error(p.dbg, PKV_DBG_LENGTH);
+    L = cap;
+  }
+  return max(L, 0);
+}
+
+__device__ __forceinline__ Item item_of(const GroupedParams& p, int i) {
+  Item it;
+  const int np = p.num_groups * p.row_blocks;
+  if (i < np) {
+    const int gi = i / p.row_blocks;
+    it.rb = i - gi * p.row_blocks;
+    it.prefix = true;
+    int b0 = __ldg(p.group_start + gi), b1 = __ldg(p.group_start + gi + 1);
+    b0 = min(max(b0, 0), p.batch);
+    b1 = min(max(b1, b0), min(p.batch, b0 + p.max_members));
+    it.lead = b0;
+    it.rows = min(kRows, (b1 - b0) * p.group - it.rb * kRows);
+    it.lo = 0;
+    it.hi = it.rows > 0 ? clamp_len(p, __ldg(p.shared_len + b0)) : 0;
+  } else {
+    const int b = i - np;
+    it.rb = 0;
+    it.prefix = false;
+    it.lead = b;
+    it.rows = p.group;
+    it.hi = clamp_len(p, __ldg(p.seq_lens + b));
+    it.lo = min(max(__ldg(p.shared_len + b), 0), it.hi);
+  }
+  it.t0 = it.lo / kTile;
+  it.n = it.hi > it.lo ? (it.hi + kTile - 1) / kTile - it.t0 : 0;
+  return it;
+}
+
+// Tiles per KV head summed over all items (warp-cooperative; every lane gets
+// the result); with `prefix`, also the exclusive prefix over items.
+__device__ __forceinline__ int total_tiles(const GroupedParams& p, int lane, int32_t* prefix) {
+  int run = 0;
+  for (int base = 0; base < p.items; base += 32) {
+    const int i = base + lane;
+    const int n = i < p.items ? item_of(p, i).n : 0;
+    int incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (prefix && i < p.items) prefix[i] = run + incl - n;
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (prefix && lane == 0) prefix[p.items] = run;
+  return run;
+}
+
+// Item holding global tile x, and the number of tiles (all KV heads) before it.
+__device__ __forceinline__ void find_item(const GroupedParams& p, int lane, int64_t x, int& i_out,
+                                          int64_t& before) {
+  const int H = p.num_kv_heads;
+  int64_t run = 0;
+  for (int base = 0; base < p.items; base += 32) {
+    const int i = base + lane;
+    const int n = i < p.items ? item_of(p, i).n : 0;
+    int incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const bool hit = i < p.items && run + (int64_t)incl * H > x;
+    const unsigned m = __ballot_sync(0xffffffffu, hit);
+    if (m) {
+      const int src = __ffs(m) - 1;
+      const int excl = __shfl_sync(0xffffffffu, incl - n, src);
+      i_out = base + src;
+      before = run + (int64_t)excl * H;
+      return;
+    }
+    run += (int64_t)__shfl_sync(0xffffffffu, incl, 31) * H;
+  }
+  i_out = p.items;
+  before = run;
+}
+
+__device__ __forceinline__ int workers_for(int64_t total, int launched) {
+  int64_t w = total / kMinTilesPerWorker;
+  if (w < 1) w = 1;
+  return (int)(w < launched ? w : launched);
+}
+
+// Cursor over the flat tile list (uniform across the warp).
+struct Cursor {
+  int i, kvh;
+  Item it;
+  int64_t seg_first;  // global index of the segment's first tile
+  int64_t t;          // global tile index
+};
+
+__device__ __forceinline__ void cursor_advance(const GroupedParams& p, Cursor& c) {
+  ++c.t;
+  if (c.t == c.seg_first + c.it.n) {
+    c.seg_first += c.it.n;
+    if (c.kvh + 1 < p.num_kv_heads) {
+      ++c.kvh;
+    } else {
+      do {
+        ++c.i;
+        if (c.i >= p.items) return;
+        c.it = item_of(p, c.i);
+      } while (c.it.n == 0);
+      c.kvh = 0;
+    }
+  }
+}
+
+// (sequence, query head) of row r of a segment.
+__device__ __forceinline__ void row_target(const GroupedParams& p, const Item& it, int kvh, int r,
+                                           int& b, int& h) {
+  if (it.prefix) {
+    const int R = it.rb * kRows + r;
+    b = it.lead + R / p.group;
+    h = kvh * p.group + R % p.group;
+  } else {
+    b = it.lead;
+    h = kvh * p.group + r;
+  }
+}
+
+// Byte offset of 16-byte chunk `c` (0..15) of row `r` in a swizzled tile of
+// `rows` rows: two 64-column halves, 128-byte rows, chunk index XOR row % 8.
+__device__ __forceinline__ uint32_t swz(int rows, int r, int c) {
+  return (uint32_t)((c >> 3) * (rows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kWarps * 32, 1)
+    grouped_decode_kernel(const __grid_constant__ CUtensorMap kmap,
+                          const __grid_constant__ CUtensorMap vmap, const GroupedParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  uint8_t* ring = smem + warp * kWarpSmem;
+  uint8_t* qs = ring + kStages * kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kWarpSmem) + warp * kStages;
+
+  const int gw = blockIdx.x * kWarps + warp;
+  const int64_t T =
+      (int64_t)total_tiles(p, lane, gw == 0 ? p.ws_prefix : nullptr) * p.num_kv_heads;
+  const int W = workers_for(T, p.workers);
+  if (gw >= W || T == 0) return;
+  const int64_t start = (int64_t)gw * T / W;
+  const int64_t end = (int64_t)(gw + 1) * T / W;
+  if (start >= end) return;
+
+  if (lane == 0) {
+    prefetch_tmap(&kmap);
+    prefetch_tmap(&vmap);
+    for (int i = 0; i < kStages; ++i) mbar_init(smem_u32(bars + i), 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+
+  Cursor cur;
+  {
+    int i;
+    int64_t before;
+    find_item(p, lane, start, i, before);
+    cur.i = i;
+    cur.it = item_of(p, i);
+    const int64_t off = start - before;
+    cur.kvh = (int)(off / cur.it.n);
+    cur.seg_first = before + (int64_t)cur.kvh * cur.it.n;
+    cur.t = start;
+  }
+  Cursor pc = cur;  // producer cursor
+
+  const int bs_mask = (1 << p.bs_shift) - 1;
+  const int box_rows = p.bs_shift >= 4 ? kTile : (1 << p.bs_shift);  // 8 or 16
+  const int pieces = kTile / box_rows;                                // 1 or 2
+  const uint64_t evict_first = policy_evict_first();
+
+  // block ids of the producer's next tile (lane 0), loaded one step ahead
+  int pid0 = 0, pid1 = 0;
+  auto load_ids = [&](const Cursor& c) {
+    if (lane != 0 || c.i >= p.items) return;
+    const int tok0 = (c.it.t0 + (int)(c.t - c.seg_first)) * kTile;
+    const int j = tok0 >> p.bs_shift;
+    const int32_t* row = p.tables + (int64_t)c.it.lead * p.max_blocks;
+    pid0 = j < p.max_blocks ? __ldg(row + j) : -1;
+    if (pieces == 2) pid1 = (j + 1 < p.max_blocks && tok0 + 8 < c.it.hi) ? __ldg(row + j + 1) : -1;
+  };
+  auto issue = [&](const Cursor& c, int stage) {
+    if (lane != 0) return;
+    const int tok0 = (c.it.t0 + (int)(c.t - c.seg_first)) * kTile;
+    const uint32_t bar = smem_u32(bars + stage);
+    const uint32_t kdst = smem_u32(ring + stage * kStageBytes);
+    const uint32_t vdst = kdst + kTileBytes;
+    int ids[2] = {pid0, pid1};
+    bool need[2];
+    uint32_t bytes = 0;
+    for (int pi = 0; pi < pieces; ++pi) {
+      const int a = tok0 + pi * box_rows;
+      need[pi] = a < c.it.hi && a + box_rows > c.it.lo;
+      if (need[pi]) {
+        if (ids[pi] < 0 || ids[pi] >= p.num_blocks) {
+          flag_error(p.dbg, PKV_DBG_BLOCK_ID);
+          ids[pi] = 0;
+        }
+        bytes += 2u * box_rows * kD * 2;
+      }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(bar, bytes);
+    for (int pi = 0; pi < pieces; ++pi) {
+      if (!need[pi]) continue;
+      const int row = ((ids[pi] * p.num_kv_heads + c.kvh) << p.bs_shift) +
+                      ((tok0 + pi * box_rows) & bs_mask);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t o = h * (kTile * 128) + pi * box_rows * 128;
+        tma_load_2d_hint(kdst + o, &kmap, h * 64, row, bar, evict_first);
+        tma_load_2d_hint(vdst + o, &vmap, h * 64, row, bar, evict_first);
+      }
+    }
+  };
+
+  const int64_t ntiles = end - start;
+  load_ids(pc);
+  int64_t issued = 0;
+  for (; issued < kStages - 1 && issued < ntiles; ++issued) {
+    issue(pc, (int)(issued % kStages));
+    cursor_advance(p, pc);
+    if (issued + 1 < ntiles) load_ids(pc);
+  }
+
+  // lane roles in the mma fragments
+  const int g4 = lane >> 2;
+  const int c4 = lane & 3;
+  const int mi = lane >> 3, mr = lane & 7;
+  const int krow = mr + ((mi & 1) << 3);   // K tile row (token) this lane addresses
+  const int kco = mi >> 1;
+  const int vtok = mr + ((mi >> 1) << 3);  // V tile row (token) this lane addresses
+  const int vco = mi & 1;
+  const int qrow = mr + ((mi >> 1) << 3);  // query row (within an n-tile pair) of this lane
+  const int qco = mi & 1;
+
+  float o[kNT][kD / 16][4];
+  float m0[kNT], m1[kNT], l0[kNT], l1[kNT];
+  int piece = 0;
+  int64_t piece_start = start;
+  int ntv = kNT;  // n-tiles holding rows of the current segment
+
+  for (int64_t k = 0; k < ntiles; ++k) {
+    if (issued < ntiles) {
+      issue(pc, (int)(issued % kStages));
+      cursor_advance(p, pc);
+      ++issued;
+      if (issued < ntiles) load_ids(pc);
+    }
+    const bool seg_begin = (k == 0) || (cur.t == cur.seg_first);
+    if (seg_begin) {
+      piece_start = cur.t;
+      ntv = (cur.it.rows + 7) >> 3;
+      // stage the segment's query rows (zero past its last row), swizzled
+      for (int x = lane; x < kRows * 16; x += 32) {
+        const int r = x >> 4, c = x & 15;
+        int4 v = make_int4(0, 0, 0, 0);
+        if (r < cur.it.rows) {
+          int b, h;
+          row_target(p, cur.it, cur.kvh, r, b, h);
+          v = __ldg(reinterpret_cast<const int4*>(p.q + ((int64_t)b * p.num_q_heads + h) * kD) +
+                    c);
+        }
+        *reinterpret_cast<int4*>(qs + swz(kRows, r, c)) = v;
+      }
+      __syncwarp();
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+#pragma unroll
+        for (int mt = 0; mt < kD / 16; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+        m0[nt] = m1[nt] = -INFINITY;
+        l0[nt] = l1[nt] = 0.f;
+      }
+    }
+
+    const int stage = (int)(k % kStages);
+    const uint32_t parity = (uint32_t)((k / kStages) & 1);
+    uint8_t* kst = ring + stage * kStageBytes;
+    const uint32_t kbase = smem_u32(kst);
+    const uint32_t vbase = kbase + kTileBytes;
+    const uint32_t qbase = smem_u32(qs);
+    if (!mbar_wait(smem_u32(bars + stage), parity)) {
+      flag_error(p.dbg, PKV_DBG_TIMEOUT);
+      return;
+    }
+    const int tok0 = (cur.it.t0 + (int)(cur.t - cur.seg_first)) * kTile;
+    const bool partial = tok0 < cur.it.lo || tok0 + kTile > cur.it.hi;
+    if (partial) {
+      // rows outside [lo, hi) may hold stale or non-finite data: zero them in V
+      for (int x = lane; x < kTile * 16; x += 32) {
+        const int r = x >> 4, c = x & 15;
+        const int pos = tok0 + r;
+        if (pos < cur.it.lo || pos >= cur.it.hi)
+          *reinterpret_cast<int4*>(kst + kTileBytes + swz(kTile, r, c)) = make_int4(0, 0, 0, 0);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+    }
+
+    // S^T (16 tokens x 32 rows) = K (16 x D) * Q^T (D x 32)
+    float s[kNT][4];
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < kD / 16; ++kk) {
+      uint32_t a[4];
+      ldmatrix_x4(a, kbase + swz(kTile, krow, 2 * kk + kco));
+#pragma unroll
+      for (int np = 0; np < kNT / 2; ++np) {
+        if (2 * np < ntv) {
+          // B fragments of n-tiles 2np, 2np+1: rows (n) x 16 columns (k) of the query tile
+          uint32_t bq[4];
+          ldmatrix_x4(bq, qbase + swz(kRows, np * 16 + qrow, 2 * kk + qco));
+          mma_bf16_16816(s[2 * np], a, bq[0], bq[1]);
+          if (2 * np + 1 < ntv) mma_bf16_16816(s[2 * np + 1], a, bq[2], bq[3]);
+        }
+      }
+    }
+    // element e of s[nt]: token g4 (+8 for e >= 2), row nt*8 + 2*c4 + (e & 1)
+    bool bad0 = false, bad1 = false;
+    if (partial) {
+      const int p0 = tok0 + g4, p1 = p0 + 8;
+      bad0 = p0 < cur.it.lo || p0 >= cur.it.hi;
+      bad1 = p1 < cur.it.lo || p1 >= cur.it.hi;
+    }
+    uint32_t pb0[kNT], pb1[kNT];
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) {
+      if (nt < ntv) {
+        float x0 = s[nt][0] * p.scale_log2, x1 = s[nt][1] * p.scale_log2;
+        float x2 = s[nt][2] * p.scale_log2, x3 = s[nt][3] * p.scale_log2;
+        if (bad0) x0 = x1 = -INFINITY;
+        if (bad1) x2 = x3 = -INFINITY;
+        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        // every tile of a segment holds a visible key: the new maxima are finite
+        const float n0 = fmaxf(m0[nt], mx0), n1 = fmaxf(m1[nt], mx1);
+        const float al0 = fast_exp2(m0[nt] - n0), al1 = fast_exp2(m1[nt] - n1);
+        m0[nt] = n0;
+        m1[nt] = n1;
+        const float p00 = fast_exp2(x0 - n0), p01 = fast_exp2(x1 - n1);
+        const float p10 = fast_exp2(x2 - n0), p11 = fast_exp2(x3 - n1);
+        l0[nt] = l0[nt] * al0 + p00 + p10;
+        l1[nt] = l1[nt] * al1 + p01 + p11;
+        if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+          for (int mt = 0; mt < kD / 16; ++mt) {
+            o[nt][mt][0] *= al0;
+            o[nt][mt][1] *= al1;
+            o[nt][mt][2] *= al0;
+            o[nt][mt][3] *= al1;
+          }
+        }
+        pb0[nt] = movmatrix_trans(pack_bf16x2(p00, p01));
+        pb1[nt] = movmatrix_trans(pack_bf16x2(p10, p11));
+      }
+    }
+    // O^T (D x 32) += V^T (D x 16 tokens) * P^T (16 x 32)
+#pragma unroll
+    for (int mt = 0; mt < kD / 16; ++mt) {
+      uint32_t a[4];
+      ldmatrix_x4_trans(a, vbase + swz(kTile, vtok, 2 * mt + vco));
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt)
+        if (nt < ntv) mma_bf16_16816(o[nt][mt], a, pb0[nt], pb1[nt]);
+    }
+    __syncwarp();
+
+    const int64_t seg_end = cur.seg_first + cur.it.n;
+    const bool piece_end = (k == ntiles - 1) || (cur.t + 1 == seg_end);
+    if (piece_end) {
+      const bool whole = (piece_start == cur.seg_first) && (cur.t + 1 == seg_end);
+      const int64_t slot = (int64_t)gw * 2 + piece;
+      const int kind = cur.it.prefix ? 0 : 1;
+      const int64_t rows_all = (int64_t)p.batch * p.num_q_heads;
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+        if (nt < ntv) {
+          float s0 = l0[nt], s1 = l1[nt];
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            s0 += __shfl_xor_sync(0xffffffffu, s0, off);
+            s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+          }
+          const float inv[2] = {1.f / s0, 1.f / s1};
+          const float ls[2] = {m0[nt] * kLn2 + logf(s0), m1[nt] * kLn2 + logf(s1)};
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int r = nt * 8 + 2 * c4 + j;
+            if (r >= cur.it.rows) continue;
+            float* dst;
+            float* dl;
+            if (whole) {
+              int b, h;
+              row_target(p, cur.it, cur.kvh, r, b, h);
+              const int64_t orow = kind * rows_all + (int64_t)b * p.num_q_heads + h;
+              dst = p.whole_o + orow * kD;
+              dl = p.whole_lse + orow;
+            } else {
+              dst = p.ws_o + (slot * kRows + r) * kD;
+              dl = p.ws_lse + slot * kRows + r;
+            }
+#pragma unroll
+            for (int mt = 0; mt < kD / 16; ++mt) {
+              dst[mt * 16 + g4] = o[nt][mt][j] * inv[j];
+              dst[mt * 16 + g4 + 8] = o[nt][mt][2 + j] * inv[j];
+            }
+            if (g4 == 0) *dl = ls[j];
+          }
+        }
+      }
+      piece = 1;  // the worker's later piece, if split, is its last: slot 1
+    }
+    cursor_advance(p, cur);
+  }
+}
+
+namespace {
+
+// Group of sequence b: the last gi with group_start[gi] <= b, by a 32-way
+// search across the warp (every lane gets the answer; -1 if b precedes all).
+__device__ __forceinline__ int find_group(const GroupedParams& p, int lane, int b) {
+  int lo = 0, hi = p.num_groups;
+  while (true) {
+    const int step = (hi - lo + 31) / 32;
+    const int idx = lo + lane * step;
+    const bool le = idx < hi && __ldg(p.group_start + idx) <= b;
+    const unsigned m = __ballot_sync(0xffffffffu, le);
+    if (!m) return -1;
+    lo += (31 - __clz(m)) * step;
+    if (step == 1) return lo;
+    hi = min(hi, lo + step);
+  }
+}
+
+// Result of segment (item i, KV head kvh) for its row r: this lane's four
+// output columns (normalised) and the LSE (-inf for an empty segment). A
+// segment one worker did whole is read from whole_o / whole_lse at
+// `whole_row`; a split one merges its workers' pieces by log-sum-exp.
+__device__ __forceinline__ float segment_result(const GroupedParams& p, int lane, int i, int kvh,
+                                                int r, int64_t whole_row, float (&acc)[4]) {
+  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+  const int H = p.num_kv_heads;
+  const int n = p.ws_prefix[i + 1] - p.ws_prefix[i];
+  if (n <= 0) return -INFINITY;
+  const int64_t T = (int64_t)p.ws_prefix[p.items] * H;
+  const int W = workers_for(T, p.workers);
+  const int64_t s0 = (int64_t)p.ws_prefix[i] * H + (int64_t)kvh * n;
+  const int64_t s1 = s0 + n;
+  auto owner = [&](int64_t x) { return (int)(((x + 1) * W - 1) / T); };
+  const int wf = owner(s0), wl = owner(s1 - 1);
+  if (wf == wl) {
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(p.whole_o + whole_row * kD) + lane);
+    acc[0] = v.x;
+    acc[1] = v.y;
+    acc[2] = v.z;
+    acc[3] = v.w;
+    return __ldcg(p.whole_lse + whole_row);
+  }
+  // slot of worker w's piece of this segment, or -1 if w has no tiles
+  auto slot_of = [&](int w) -> int64_t {
+    const int64_t st = (int64_t)w * T / W, en = (int64_t)(w + 1) * T / W;
+    if (st == en) return -1;
+    return (int64_t)w * 2 + ((w == wf && st < s0) ? 1 : 0);
+  };
+  float m = -INFINITY, sum = 0.f;
+  for (int base = wf; base <= wl; base += 32) {
+    const int w = base + lane;
+    float x = -INFINITY;
+    if (w <= wl) {
+      const int64_t sl = slot_of(w);
+      if (sl >= 0) x = __ldcg(p.ws_lse + sl * kRows + r);
+    }
+    float mx = x;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float nm = fmaxf(m, mx);
+    float e = (x == -INFINITY) ? 0.f : __expf(x - nm);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+    sum = (m == -INFINITY ? 0.f : sum * __expf(m - nm)) + e;
+    m = nm;
+  }
+  const float lse = m + logf(sum);
+  for (int base = wf; base <= wl; base += 32) {
+    const int w = base + lane;
+    int64_t sl = -1;
+    float wgt = 0.f;
+    if (w <= wl) {
+      sl = slot_of(w);
+      if (sl >= 0) wgt = __expf(__ldcg(p.ws_lse + sl * kRows + r) - lse);
+    }
+    const int cnt = min(32, wl - base + 1);
+    for (int j = 0; j < cnt; ++j) {
+      const float wj = __shfl_sync(0xffffffffu, wgt, j);
+      const int64_t sj = __shfl_sync(0xffffffffu, sl, j);
+      if (sj < 0) continue;
+      const float4 v =
+          __ldcg(reinterpret_cast<const float4*>(p.ws_o + (sj * kRows + r) * kD) + lane);
+      acc[0] += wj * v.x;
+      acc[1] += wj * v.y;
+      acc[2] += wj * v.z;
+      acc[3] += wj * v.w;
+    }
+  }
+  return lse;
+}
+
+}  // namespace
+
+// One warp per (sequence, query head): prefix result and own-key result,
+// each merged from its pieces, then merged with each other.
+__global__ void __launch_bounds__(128) grouped_combine_kernel(const GroupedParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int64_t rows_all = (int64_t)p.batch * p.num_q_heads;
+  if (row >= rows_all) return;
+  const int b = (int)(row / p.num_q_heads);
+  const int h = (int)(row % p.num_q_heads);
+  const int kvh = h / p.group, hh = h % p.group;
+  if (row == 0 && lane == 0 &&
+      (p.group_start[0] != 0 || p.group_start[p.num_groups] != p.batch))
+    flag_error(p.dbg, PKV_DBG_LENGTH);
+
+  // the sequence's group and its row in the group's prefix items
+  float op[4], os[4];
+  float lp = -INFINITY;
+  const int gi = find_group(p, lane, b);
+  bool ok = gi >= 0 && gi < p.num_groups;
+  int b0 = 0;
+  if (ok) {
+    b0 = __ldg(p.group_start + gi);
+    const int b1 = __ldg(p.group_start + gi + 1);
+    const int sl = __ldg(p.shared_len + b);
+    ok = b0 >= 0 && b < b1 && b1 - b0 <= p.max_members && sl == __ldg(p.shared_len + b0) &&
+         sl >= 0 && sl <= __ldg(p.seq_lens + b);
+  }
+  if (!ok) {
+    if (lane == 0) flag_error(p.dbg, PKV_DBG_LENGTH);
+    op[0] = op[1] = op[2] = op[3] = 0.f;
+  } else {
+    const int R = (b - b0) * p.group + hh;
+    lp = segment_result(p, lane, gi * p.row_blocks + R / kRows, kvh, R % kRows, row, op);
+  }
+  const float ls = segment_result(p, lane, p.num_groups * p.row_blocks + b, kvh, hh,
+                                  rows_all + row, os);
+  const float m = fmaxf(lp, ls);
+  float v[4] = {0.f, 0.f, 0.f, 0.f};
+  float lse = -INFINITY;
+  if (m != -INFINITY) {
+    const float wp = lp == -INFINITY ? 0.f : __expf(lp - m);
+    const float ws = ls == -INFINITY ? 0.f : __expf(ls - m);
+    const float inv = 1.f / (wp + ws);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = (wp * op[j] + ws * os[j]) * inv;
+    lse = m + logf(wp + ws);
+  }
+  uint2 packed;
+  packed.x = pack_bf16x2(v[0], v[1]);
+  packed.y = pack_bf16x2(v[2], v[3]);
+  reinterpret_cast<uint2*>(p.out + row * kD)[lane] = packed;
+  if (p.lse && lane == 0) p.lse[row] = lse;
+}
+
+namespace {
+
+// Workspace: pieces (2 per worker), whole-segment results (prefix and own
+// keys per (sequence, head)), tile prefix over items (at most 5 * batch items:
+// groups * row blocks <= 4 * batch when max_group_size * g <= 128).
+struct Layout {
+  size_t ws_o, ws_lse, whole_o, whole_lse, prefix, total;
+};
+
+Layout layout(int32_t batch, int32_t num_q_heads) {
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-  Layout l;
-  l.dec = up(decode_workspace_size(batch, num_q_heads, c));
+  const size_t workers = (size_t)device_sm_count() * kWarps;
   const size_t rows = (size_t)batch * num_q_heads;
-  l.part_o = l.dec;
-  l.part_lse = l.part_o + up(rows * kD * 4);
-  l.lse_s = l.part_lse + up(rows * 4);
-  l.total = l.lse_s + up(rows * 4);
+  Layout l;
+  l.ws_o = 0;
+  l.ws_lse = l.ws_o + up(2 * workers * kRows * kD * 4);
+  l.whole_o = l.ws_lse + up(2 * workers * kRows * 4);
+  l.whole_lse = l.whole_o + up(2 * rows * kD * 4);
+  l.prefix = l.whole_lse + up(2 * rows * 4);
+  l.total = l.prefix + up(((size_t)5 * batch + 1) * 4);
   return l;
 }
 
@@ -89,7 +713,7 @@ PKV_API size_t paged_attention_decode_shared_prefix_workspace_size(int32_t batch
   if (check_cache(cache, "paged_attention_decode_shared_prefix_workspace_size") != PKV_OK)
     return 0;
   if (batch <= 0 || num_q_heads <= 0 || num_q_heads % cache.num_kv_heads) return 0;
-  return layout(batch, num_q_heads, cache).total;
+  return layout(batch, num_q_heads).total;
 }
 
 PKV_API int paged_attention_decode_shared_prefix(
@@ -105,6 +729,8 @@ PKV_API int paged_attention_decode_shared_prefix(
   if (int st = check_mask(mask, fn)) return st;
   if (cache.dtype != PKV_BF16 || cache.head_dim != kD)
     return fail(PKV_ERR_UNSUPPORTED, "%s: bf16 pools with head_dim 128 only", fn);
+  if (cache.block_size < 8)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: block_size must be >= 8", fn);
   if (mask.kind == PKV_MASK_SLIDING)
     return fail(PKV_ERR_UNSUPPORTED, "%s: mask must be none or causal", fn);
   if (batch < 0 || max_blocks_per_seq <= 0)
@@ -112,46 +738,92 @@ PKV_API int paged_attention_decode_shared_prefix(
   if (num_q_heads <= 0 || num_q_heads % cache.num_kv_heads)
     return fail(PKV_ERR_INVALID_ARG, "%s: num_q_heads %d not a multiple of num_kv_heads %d", fn,
                 num_q_heads, cache.num_kv_heads);
+  const int g = num_q_heads / cache.num_kv_heads;
+  if (g > kRows)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: %d query heads per KV head (at most %d)", fn, g, kRows);
   if (!(scale == scale)) return fail(PKV_ERR_INVALID_ARG, "%s: scale is NaN", fn);
   if (batch == 0) return PKV_OK;
-  if (num_groups <= 0 || max_group_size <= 0)
-    return fail(PKV_ERR_INVALID_ARG, "%s: num_groups and max_group_size must be positive", fn);
-  const int g = num_q_heads / cache.num_kv_heads;
+  if (num_groups <= 0 || num_groups > batch || max_group_size <= 0)
+    return fail(PKV_ERR_INVALID_ARG, "%s: need 1 <= num_groups <= batch and max_group_size >= 1",
+                fn);
   if (max_group_size > batch) max_group_size = batch;  // no group is larger than the batch
   if ((int64_t)max_group_size * g > 128)
-    return fail(PKV_ERR_UNSUPPORTED, "%s: max_group_size * (num_q_heads / num_kv_heads) = %lld"
-                " exceeds 128 rows", fn, (long long)max_group_size * g);
+    return fail(PKV_ERR_UNSUPPORTED,
+                "%s: max_group_size * (num_q_heads / num_kv_heads) = %lld exceeds 128", fn,
+                (long long)max_group_size * g);
   if (!q || !k_cache || !v_cache || !block_tables || !seq_lens || !group_start || !shared_len ||
       !out || !workspace)
     return fail(PKV_ERR_INVALID_ARG, "%s: null pointer", fn);
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
       !aligned16(workspace))
     return fail(PKV_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", fn);
-  const Layout l = layout(batch, num_q_heads, cache);
+  const Layout l = layout(batch, num_q_heads);
   if (workspace_bytes < l.total)
     return fail(PKV_ERR_WORKSPACE_TOO_SMALL, "%s: workspace needs %zu bytes, got %zu", fn, l.total,
                 workspace_bytes);
+
+  const int sms = device_sm_count();
+  const size_t smem = (size_t)kWarps * kWarpSmem + kWarps * kStages * 8 + 1024;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(grouped_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return check_launch("paged_attention_decode_shared_prefix: smem attribute");
+    attr_set[dev] = true;
+  }
+  const int box_rows = cache.block_size >= kTile ? kTile : cache.block_size;
+  const int64_t pool_rows = (int64_t)cache.num_blocks * cache.num_kv_heads * cache.block_size;
+  alignas(64) CUtensorMap kmap, vmap;
+  if (!make_pool_tensor_map(&kmap, k_cache, pool_rows, kD, box_rows) ||
+      !make_pool_tensor_map(&vmap, v_cache, pool_rows, kD, box_rows))
+    return fail(PKV_ERR_CUDA, "%s: tensor map encoding failed", fn);
+
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* part_o = reinterpret_cast<float*>(ws + l.part_o);
-  float* part_lse = reinterpret_cast<float*>(ws + l.part_lse);
-  float* lse_s = reinterpret_cast<float*>(ws + l.lse_s);
+  GroupedParams p = {};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.tables = block_tables;
+  p.max_blocks = max_blocks_per_seq;
+  p.seq_lens = seq_lens;
+  p.group_start = group_start;
+  p.shared_len = shared_len;
+  p.batch = batch;
+  p.num_groups = num_groups;
+  p.max_members = max_group_size;
+  p.row_blocks = (max_group_size * g + kRows - 1) / kRows;
+  p.items = num_groups * p.row_blocks + batch;
+  p.num_kv_heads = cache.num_kv_heads;
+  p.group = g;
+  p.num_q_heads = num_q_heads;
+  p.bs_shift = log2_int(cache.block_size);
+  p.num_blocks = cache.num_blocks;
+  p.scale_log2 = scale * kLog2e;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.ws_o = reinterpret_cast<float*>(ws + l.ws_o);
+  p.ws_lse = reinterpret_cast<float*>(ws + l.ws_lse);
+  p.whole_o = reinterpret_cast<float*>(ws + l.whole_o);
+  p.whole_lse = reinterpret_cast<float*>(ws + l.whole_lse);
+  p.ws_prefix = reinterpret_cast<int32_t*>(ws + l.prefix);
+  p.workers = sms * kWarps;
+  p.dbg = dbg_err;
+
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // 1. shared prefixes, once per (group, KV head)
-  GroupPrefixArgs ga{q,        k_cache,        v_cache,    cache,  block_tables, max_blocks_per_seq,
-                     seq_lens, batch,          num_q_heads, scale, group_start,  num_groups,
-                     max_group_size, shared_len, part_o,    part_lse, dbg_err,   s};
-  if (int st = launch_prefix_groups(ga)) return st;
-  // 2. each sequence's own keys, from its shared length on
-  DecodeArgs a{q,        k_cache, v_cache,     cache, block_tables, max_blocks_per_seq,
-               seq_lens, batch,   num_q_heads, scale, mask,         out,
-               lse_s,    ws,      l.dec,       dbg_err, s};
-  a.key_start = shared_len;
-  if (int st = launch_decode(a)) return st;
-  // 3. merge in place
+  grouped_decode_kernel<<<sms, kWarps * 32, smem, s>>>(kmap, vmap, p);
+  if (int st = check_launch(fn)) return st;
   const int64_t rows = (int64_t)batch * num_q_heads;
-  shared_prefix_merge_kernel<<<(unsigned)((rows + 3) / 4), 128, 0, s>>>(
-      static_cast<__nv_bfloat16*>(out), lse, part_o, part_lse, lse_s, shared_len, batch,
-      num_q_heads);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((rows + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, grouped_combine_kernel, p);
   return check_launch(fn);
 }
 

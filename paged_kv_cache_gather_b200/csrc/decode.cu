@@ -63,7 +63,6 @@ struct DecodeParams {
   int32_t* ws_prefix;  // [batch + 1] tiles per KV head before sequence b
   int32_t workers;     // warps launched
   int32_t* dbg;
-  const int32_t* key_start;  // [batch] or null: keys below it are left out (shared-prefix decode)
 };
 
 // Visible range and tile span of sequence b.
@@ -83,7 +82,6 @@ __device__ __forceinline__ SeqSpan seq_span(const DecodeParams& p, int b) {
     L = cap;
   }
   decode_key_range(p.mask_kind, p.window, p.window_per_seq, b, L, s.lo, s.hi);
-  if (p.key_start) s.lo = max(s.lo, min(__ldg(p.key_start + b), s.hi));
   s.t0 = s.lo / kTile;
   s.n = s.hi > s.lo ? (s.hi + kTile - 1) / kTile - s.t0 : 0;
   return s;
@@ -695,7 +693,7 @@ int launch_bf16_impl(const DecodeArgs& a) {
     return fail(PKV_ERR_CUDA, "paged_attention_decode: tensor map encoding failed");
 
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
-  DecodeParams p = {};
+  DecodeParams p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.tables = a.tables;
   p.max_blocks = a.max_blocks;
@@ -719,7 +717,6 @@ int launch_bf16_impl(const DecodeArgs& a) {
   p.ws_prefix = reinterpret_cast<int32_t*>(ws + o_bytes + l_bytes);
   p.workers = workers;
   p.dbg = a.dbg;
-  p.key_start = a.key_start;
 
   decode_bf16_kernel<D, NSTAGE, WPC><<<sms, WPC * 32, smem, a.stream>>>(kmap, vmap, p);
   if (int st = check_launch("paged_attention_decode")) return st;

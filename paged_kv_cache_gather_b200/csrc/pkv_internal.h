@@ -62,7 +62,6 @@ struct DecodeArgs {
   size_t workspace_bytes;
   int32_t* dbg;
   cudaStream_t stream;
-  const int32_t* key_start = nullptr;  // per-sequence first key (shared-prefix decode), or null
 };
 
 size_t decode_workspace_size(int32_t batch, int32_t num_q_heads, const pkv_cache_desc& c);
@@ -92,30 +91,6 @@ struct PrefillArgs {
 
 int launch_prefill(const PrefillArgs& a);
 
-// Shared-prefix part of a grouped decode: per (group, KV head), every member's
-// query heads over the group's shared prefix; float32 partials per
-// (sequence, query head) into part_o [batch*Hq, D] and part_lse [batch*Hq].
-struct GroupPrefixArgs {
-  const void* q;  // [batch, Hq, D] bf16
-  const void* k_cache;
-  const void* v_cache;
-  pkv_cache_desc cache;
-  const int32_t* tables;
-  int32_t max_blocks;
-  const int32_t* seq_lens;  // [batch], to check shared_len <= seq_len on the device
-  int32_t batch;
-  int32_t num_q_heads;
-  float scale;
-  const int32_t* group_start;
-  int32_t num_groups;
-  int32_t max_group_size;
-  const int32_t* shared_len;
-  float* part_o;
-  float* part_lse;
-  int32_t* dbg;
-  cudaStream_t stream;
-};
-int launch_prefix_groups(const GroupPrefixArgs& a);
 
 // Encodes a 2-D bf16 tensor map over a pool viewed as [rows, head_dim] with a
 // [box_rows, 64]-element box and 128-byte swizzle. Returns false on failure.

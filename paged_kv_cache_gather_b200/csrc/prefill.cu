@@ -77,16 +77,6 @@ struct PrefillParams {
   __nv_bfloat16* out;
   float* lse;
   int32_t* dbg;
-  // group mode (shared-prefix decode): a unit is (group, KV head); its query
-  // tile holds every member's query heads of that KV head (row = member * g +
-  // head), its keys are the group's shared prefix, and it writes normalised
-  // float32 partial outputs and LSEs per (sequence, query head)
-  const int32_t* group_start;  // [num_groups + 1]: members are batch entries [start, next)
-  const int32_t* shared_len;   // [batch]: shared prefix length of each sequence
-  int32_t num_groups;
-  int32_t group_rows;          // rows the group query box loads (max members * g)
-  float* part_o;               // [batch * Hq, D]
-  float* part_lse;             // [batch * Hq]
 };
 
 struct SmemLayout {
@@ -131,39 +121,9 @@ __device__ __forceinline__ int window_of(const PrefillParams& p, int b) {
   return p.window_per_seq ? p.window_per_seq[b] : p.window;
 }
 
-template <bool kGroup>
 __device__ __forceinline__ Unit unit_of(const PrefillParams& p, const int32_t* qoff, int max_qt,
                                         int64_t u) {
   Unit x;
-  if (kGroup) {
-    const int gi = (int)(u / p.num_kv_heads);
-    x.kvh = (int)(u % p.num_kv_heads);
-    x.hp = 0;
-    x.qt = 0;
-    int b0 = p.group_start[gi], b1 = p.group_start[gi + 1];
-    if (b0 < 0 || b1 < b0 || b1 > p.batch || b1 - b0 > p.group_rows / p.group) {
-      flag_error(p.dbg, PKV_DBG_LENGTH);
-      b0 = min(max(b0, 0), p.batch);
-      b1 = min(max(b1, b0), min(p.batch, b0 + p.group_rows / p.group));
-    }
-    x.b = b0;                                      // first member: its table holds the prefix
-    x.qoff = x.b;
-    x.Q = b1 - b0;                                 // members
-    int C = x.Q > 0 ? p.shared_len[x.b] : 0;
-    const int cap = p.max_blocks << p.bs_shift;
-    if (C > cap) {
-      flag_error(p.dbg, PKV_DBG_LENGTH);
-      C = cap;
-    }
-    x.C = max(C, 0);
-    x.window = 0;
-    x.valid = x.Q > 0 && x.C > 0;
-    x.ctx_lo = 0;
-    x.n_ctx = (x.C + kN - 1) / kN;
-    x.ch_lo = 0;
-    x.n_ch = 0;
-    return x;
-  }
   const int64_t per_qt = (int64_t)p.batch * p.num_kv_heads * p.pairs;
   const int qt_rev = (int)(u / per_qt);
   int64_t rem = u - (int64_t)qt_rev * per_qt;
@@ -260,9 +220,6 @@ struct Maps {
   CUtensorMap vpool;
 };
 
-// kGroup selects group mode (shared-prefix decode) at compile time, so the
-// prefill instance carries none of its code.
-template <bool kGroup>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ Maps maps, const PrefillParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -307,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // exclusive prefix of q_lens and the largest number of query tiles
     int run = 0, mq = 0;
-    for (int base = 0; !kGroup && base < p.batch; base += 32) {
+    for (int base = 0; base < p.batch; base += 32) {
       const int b = base + lane;
       int q = b < p.batch ? max(0, p.q_lens[b]) : 0;
       mq = max(mq, (q + kM - 1) / kM);
@@ -323,47 +280,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int o = 16; o; o >>= 1) mq = max(mq, __shfl_xor_sync(0xffffffffu, mq, o));
     if (lane == 0) {
-      if (!kGroup) qoff[p.batch] = run;
+      qoff[p.batch] = run;
       *max_qt_s = mq;
-      if (!kGroup && run != p.total_q && blockIdx.x == 0)
-        flag_error(p.dbg, PKV_DBG_QLEN_SUM);
-    }
-    if (kGroup) {
-      // groups must tile the batch in order, and every member shares the
-      // leader's prefix length, which may not pass its own sequence length
-      for (int gi = blockIdx.x; gi < p.num_groups; gi += gridDim.x) {
-        const int b0 = p.group_start[gi], b1 = p.group_start[gi + 1];
-        bool bad = (gi == 0 && b0 != 0) || (gi == p.num_groups - 1 && b1 != p.batch) ||
-                   b0 < 0 || b1 <= b0 || b1 > p.batch || b1 - b0 > p.group_rows / p.group;
-        if (!bad) {
-          const int C = p.shared_len[b0];
-          for (int m = b0 + lane; m < b1; m += 32)
-            bad |= p.shared_len[m] != C || C < 0 || C > p.ctx_lens[m];
-        }
-        if (__any_sync(0xffffffffu, bad) && lane == 0) flag_error(p.dbg, PKV_DBG_LENGTH);
-      }
+      if (run != p.total_q && blockIdx.x == 0) flag_error(p.dbg, PKV_DBG_QLEN_SUM);
     }
   } else if (warp == 9) {
     tc::tmem_alloc(smem_u32(tmem_slot), 512);
     tc::tmem_relinquish();
   }
-  if (kGroup && warp < 8) {
-    // a group's query box fills only its first rows: the rest of the tile is
-    // zero, so those rows compute harmless finite values that are never stored
-    for (int i = tid; i < kTileBytes / 16; i += 256)
-      *reinterpret_cast<int4*>(smem + L::kQ0 + i * 16) = make_int4(0, 0, 0, 0);
-    fence_proxy_async_smem();
-  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int max_qt = kGroup ? 1 : *max_qt_s;
-  const int64_t num_units = kGroup
-                                ? (int64_t)p.num_groups * p.num_kv_heads
-                                : (int64_t)max_qt * p.batch * p.num_kv_heads * p.pairs;
-  const uint32_t q_bytes =
-      kGroup ? 2u * p.group_rows * 128u : (p.two_heads ? 2u : 1u) * kTileBytes;
+  const int max_qt = *max_qt_s;
+  const int64_t num_units = (int64_t)max_qt * p.batch * p.num_kv_heads * p.pairs;
+  const uint32_t q_bytes = (p.two_heads ? 2u : 1u) * kTileBytes;
 
   if (warp == 8) {
     // ================================================================ TMA producer
@@ -392,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int unit_k = 0;
     uint32_t cnt = 0;  // tiles issued (K and V rings advance together)
     for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
-      const Unit x = unit_of<kGroup>(p, qoff, max_qt, u);
+      const Unit x = unit_of(p, qoff, max_qt, u);
       if (!x.valid) continue;
       const int h0 = x.kvh * p.group + x.hp * (p.two_heads ? 2 : 1);
       const int n = x.n();
@@ -401,18 +332,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (unit_k > 0 && !wait_or_flag(bar(BAR_Q_EMPTY), (unit_k - 1) & 1, p.dbg, abort_flag)) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(BAR_Q_FULL), q_bytes);
-        if (kGroup) {
-          // rows (member, head): box {64, g, max members} at (kv head's first head, leader)
+        const int row0 = x.qoff + x.qt * kM;
+        for (int hh = 0; hh < (p.two_heads ? 2 : 1); ++hh)
           for (int half = 0; half < 2; ++half)
-            tma_load_3d(smem_u32(smem + L::kQ0 + half * kHalfBytes), &maps.q, half * 64,
-                        x.kvh * p.group, x.b, bar(BAR_Q_FULL));
-        } else {
-          const int row0 = x.qoff + x.qt * kM;
-          for (int hh = 0; hh < (p.two_heads ? 2 : 1); ++hh)
-            for (int half = 0; half < 2; ++half)
-              tma_load_3d(smem_u32(smem + (hh ? L::kQ1 : L::kQ0) + half * kHalfBytes), &maps.q,
-                          half * 64, h0 + hh, row0, bar(BAR_Q_FULL));
-        }
+            tma_load_3d(smem_u32(smem + (hh ? L::kQ1 : L::kQ0) + half * kHalfBytes), &maps.q,
+                        half * 64, h0 + hh, row0, bar(BAR_Q_FULL));
       }
       bool ok = true;
       for (int j = 0; j < n; ++j, ++cnt) {
@@ -504,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mma_ts(d, p_tmem + kk * 8, dv + (uint64_t)(kk * (2048 >> 4)), idesc_o, acc || kk > 0);
     };
     for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
-      const Unit x = unit_of<kGroup>(p, qoff, max_qt, u);
+      const Unit x = unit_of(p, qoff, max_qt, u);
       if (!x.valid) continue;
       const int n = x.n();
       if (!wait_or_flag(bar(BAR_Q_FULL), unit_k & 1, p.dbg, abort_flag)) break;
@@ -600,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int unit_k = 0;
     uint32_t s_cnt = 0;
     for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
-      const Unit x = unit_of<kGroup>(p, qoff, max_qt, u);
+      const Unit x = unit_of(p, qoff, max_qt, u);
       if (!x.valid) continue;
       if (hsel == 1 && !p.two_heads) {
         ++unit_k;
@@ -719,30 +643,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue: O / l -> bf16, lse
       if (!wait_or_flag(bar(BAR_O_FULL + hsel), unit_k & 1, p.dbg, abort_flag, true)) break;
       tc::fence_after_sync();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      if (kGroup) {
-        // row = member * g + head: normalised float32 partial and its LSE
-        const bool valid_row = row < x.Q * p.group;
-        const int bm = x.b + row / p.group;
-        const int64_t orow = (int64_t)bm * p.num_q_heads + x.kvh * p.group + row % p.group;
-        float* dstf = p.part_o + orow * kD;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tc::ld32(O + c * 32, o);
-          tc::wait_ld();
-          if (valid_row) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(dstf + c * 32 + i) =
-                  make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
-                              __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-          }
-        }
-        if (valid_row) p.part_lse[orow] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
-      } else {
       const int h = x.kvh * p.group + x.hp * (p.two_heads ? 2 : 1) + hsel;
       const bool valid_row = i_row < x.Q && x.qoff + i_row < p.total_q;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* dst = p.out + ((int64_t)(x.qoff + i_row) * p.num_q_heads + h) * kD;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -764,7 +667,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (valid_row && p.lse)
         p.lse[(int64_t)(x.qoff + i_row) * p.num_q_heads + h] =
             l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
-      }
       tc::fence_before_sync();
       mbar_arrive(bar(BAR_O_FREE + hsel));
       ++unit_k;
@@ -779,78 +681,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Allows the kernel's dynamic shared memory (once per device and instance).
-template <bool kGroup>
-int set_prefill_smem_attr() {
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    const size_t max_smem = SmemLayout::kQoff + (size_t)(kMaxBatch + 1) * 4 + 1024;
-    if (cudaFuncSetAttribute(prefill_kernel<kGroup>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)max_smem) != cudaSuccess)
-      return check_launch("paged_attention_prefill: smem attribute");
-    attr_set[dev] = true;
-  }
-  return PKV_OK;
-}
-
 bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
               const uint64_t* strides_bytes, const uint32_t* box) {
   return make_tensor_map_bf16(m, base, rank, dims, strides_bytes, box);
 }
 
 }  // namespace
-
-int launch_prefix_groups(const GroupPrefixArgs& a) {
-  const char* fn = "paged_attention_decode_shared_prefix";
-  const int Hkv = a.cache.num_kv_heads;
-  const int g = a.num_q_heads / Hkv;
-  PrefillParams p = {};
-  p.tables = a.tables;
-  p.max_blocks = a.max_blocks;
-  p.batch = a.batch;
-  p.total_q = a.batch;
-  p.num_q_heads = a.num_q_heads;
-  p.num_kv_heads = Hkv;
-  p.group = g;
-  p.two_heads = 0;
-  p.pairs = 1;
-  p.bs_shift = log2_int(a.cache.block_size);
-  p.box_rows = a.cache.block_size < 16 ? a.cache.block_size : 16;
-  p.num_blocks = a.cache.num_blocks;
-  const int64_t pool_rows = (int64_t)a.cache.num_blocks * Hkv * a.cache.block_size;
-  p.pool_rows = (int32_t)pool_rows;
-  p.scale_log2 = a.scale * kLog2e;
-  p.mask_kind = PKV_MASK_NONE;  // every member sits past the whole prefix
-  p.ctx_lens = a.seq_lens;      // group mode: only checked against shared_len
-  p.dbg = a.dbg;
-  p.group_start = a.group_start;
-  p.shared_len = a.shared_len;
-  p.num_groups = a.num_groups;
-  p.group_rows = a.max_group_size * g;
-  p.part_o = a.part_o;
-  p.part_lse = a.part_lse;
-  alignas(64) Maps maps;
-  {
-    const uint64_t dq[3] = {(uint64_t)kD, (uint64_t)a.num_q_heads, (uint64_t)a.batch};
-    const uint64_t sq[2] = {(uint64_t)kD * 2, (uint64_t)a.num_q_heads * kD * 2};
-    const uint32_t boxq[3] = {64, (uint32_t)g, (uint32_t)a.max_group_size};
-    const uint64_t dp[2] = {(uint64_t)kD, (uint64_t)pool_rows};
-    const uint64_t sp[1] = {(uint64_t)kD * 2};
-    const uint32_t boxp[2] = {64, (uint32_t)p.box_rows};
-    if (!make_map(&maps.q, a.q, 3, dq, sq, boxq) ||
-        !make_map(&maps.kpool, a.k_cache, 2, dp, sp, boxp) ||
-        !make_map(&maps.vpool, a.v_cache, 2, dp, sp, boxp))
-      return fail(PKV_ERR_CUDA, "%s: tensor map encoding failed", fn);
-    maps.knew = maps.kpool;  // no chunk keys in group mode
-    maps.vnew = maps.vpool;
-  }
-  const size_t smem = SmemLayout::kQoff + 16 + 1024;  // no per-sequence offsets in group mode
-  if (int st = set_prefill_smem_attr<true>()) return st;
-  prefill_kernel<true><<<device_sm_count(), kThreads, smem, a.stream>>>(maps, p);
-  return check_launch(fn);
-}
 
 int launch_prefill(const PrefillArgs& a) {
   const char* fn = "paged_attention_prefill";
@@ -864,7 +700,7 @@ int launch_prefill(const PrefillArgs& a) {
     return fail(PKV_ERR_UNSUPPORTED, "%s: batch %d > %d", fn, a.batch, kMaxBatch);
   const int Hkv = a.cache.num_kv_heads;
   const int g = a.num_q_heads / Hkv;
-  PrefillParams p = {};
+  PrefillParams p;
   p.tables = a.tables;
   p.max_blocks = a.max_blocks;
   p.ctx_lens = a.ctx_lens;
@@ -907,9 +743,18 @@ int launch_prefill(const PrefillArgs& a) {
       return fail(PKV_ERR_CUDA, "%s: tensor map encoding failed", fn);
   }
   const size_t smem = SmemLayout::kQoff + (size_t)(a.batch + 1) * 4 + 1024;
-  if (int st = set_prefill_smem_attr<false>()) return st;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    const size_t max_smem = SmemLayout::kQoff + (size_t)(kMaxBatch + 1) * 4 + 1024;
+    if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)max_smem) != cudaSuccess)
+      return check_launch("paged_attention_prefill: smem attribute");
+    attr_set[dev] = true;
+  }
   const int grid = device_sm_count();
-  prefill_kernel<false><<<grid, kThreads, smem, a.stream>>>(maps, p);
+  prefill_kernel<<<grid, kThreads, smem, a.stream>>>(maps, p);
   return check_launch(fn);
 }
 

@@ -90,6 +90,14 @@ def test_largest_group(cuda_device):
     check(case, cuda_device)
 
 
+def test_two_row_blocks(cuda_device):
+    # 16 members x 4 heads = 64 rows: the prefix is attended in two 32-row blocks
+    rng = np.random.default_rng(6)
+    case = ragged("rows64", 6, group_sizes=[16, 16, 3], prefix_lens=[700, 1400, 5],
+                  suffix_lens=rng.integers(0, 50, size=35).tolist(), peaky=True)
+    check(case, cuda_device)
+
+
 def test_group_too_large_rejected(cuda_device):
     case = ragged("group33", 4, group_sizes=[33], prefix_lens=[64], suffix_lens=[1] * 33)
     with pytest.raises(PagedKVError):
