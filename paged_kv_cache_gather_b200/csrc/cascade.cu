@@ -604,17 +604,29 @@ __device__ __forceinline__ float segment_result(const GroupedParams& p, int lane
       sl = slot_of(w);
       if (sl >= 0) wgt = __expf(__ldcg(p.ws_lse + sl * kRows + r) - lse);
     }
+    // eight pieces' loads in flight at a time (the loop is latency-bound)
     const int cnt = min(32, wl - base + 1);
-    for (int j = 0; j < cnt; ++j) {
-      const float wj = __shfl_sync(0xffffffffu, wgt, j);
-      const int64_t sj = __shfl_sync(0xffffffffu, sl, j);
-      if (sj < 0) continue;
-      const float4 v =
-          __ldcg(reinterpret_cast<const float4*>(p.ws_o + (sj * kRows + r) * kD) + lane);
-      acc[0] += wj * v.x;
-      acc[1] += wj * v.y;
-      acc[2] += wj * v.z;
-      acc[3] += wj * v.w;
+    for (int j0 = 0; j0 < cnt; j0 += 8) {
+      float4 v[8];
+      float wv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u;
+        const float wj = __shfl_sync(0xffffffffu, wgt, j & 31);
+        const int64_t sj = __shfl_sync(0xffffffffu, sl, j & 31);
+        const bool use = j < cnt && sj >= 0;
+        wv[u] = use ? wj : 0.f;
+        v[u] = use ? __ldcg(reinterpret_cast<const float4*>(p.ws_o + (sj * kRows + r) * kD) +
+                            lane)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        acc[0] += wv[u] * v[u].x;
+        acc[1] += wv[u] * v[u].y;
+        acc[2] += wv[u] * v[u].z;
+        acc[3] += wv[u] * v[u].w;
+      }
     }
   }
   return lse;

@@ -549,22 +549,35 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
       sl = slot_of(w);
       if (sl >= 0) wgt = __expf(__ldcg(p.ws_lse + sl * p.group + h) - lse);
     }
+    // eight pieces' loads in flight at a time (the loop is latency-bound)
     const int cnt = min(32, wl - base + 1);
-    for (int j = 0; j < cnt; ++j) {
-      const float wj = __shfl_sync(0xffffffffu, wgt, j);
-      const int64_t sj = __shfl_sync(0xffffffffu, sl, j);
-      if (sj < 0) continue;
-      const float* src = p.ws_o + (sj * p.group + h) * D + lane * V;
-      if constexpr (V == 4) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
-        acc[0] += wj * v.x;
-        acc[1] += wj * v.y;
-        acc[2] += wj * v.z;
-        acc[3] += wj * v.w;
-      } else {
+    for (int j0 = 0; j0 < cnt; j0 += 8) {
+      float v[8][V];
+      float wv[8];
 #pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] += wj * __ldcg(src + i);
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u;
+        const float wj = __shfl_sync(0xffffffffu, wgt, j & 31);
+        const int64_t sj = __shfl_sync(0xffffffffu, sl, j & 31);
+        const bool use = j < cnt && sj >= 0;
+        wv[u] = use ? wj : 0.f;
+        const float* src = p.ws_o + ((use ? sj : 0) * p.group + h) * D + lane * V;
+        if constexpr (V == 4) {
+          const float4 x = use ? __ldcg(reinterpret_cast<const float4*>(src))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[u][0] = x.x;
+          v[u][1] = x.y;
+          v[u][2] = x.z;
+          v[u][3] = x.w;
+        } else {
+#pragma unroll
+          for (int i = 0; i < V; ++i) v[u][i] = use ? __ldcg(src + i) : 0.f;
+        }
       }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] += wv[u] * v[u][i];
     }
   }
 #pragma unroll
