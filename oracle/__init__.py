@@ -32,6 +32,9 @@ from .attention64 import (  # noqa: F401
     MASK_NONE,
     MASK_CAUSAL,
     MASK_SLIDING,
+    MASK_PREFIX_LM,
+    MASK_DOCUMENT,
+    document_of,
     visible,
     resolve_block_table,
     masked_attention,

@@ -15,9 +15,14 @@ Conventions (readings of the pages, listed with reasons in the design notes):
 * A slot is ``block * block_size + row``; appending a token writes its K/V to
   that slot and moves nothing else (same page, the section on dynamic growth).
 * Masks follow FlexAttention's ``mask_mod(b, h, q_idx, kv_idx)`` idea ("Paged
-  Attention Meets FlexAttention", abstract): none, causal (``kv <= q``), and
+  Attention Meets FlexAttention", abstract): none, causal (``kv <= q``),
   sliding window W (causal and ``q - kv < W``, i.e. exactly W keys including
-  the query's own position). A window ``<= 0`` means causal only.
+  the query's own position; a window ``<= 0`` means causal only; the window
+  may be per sequence or per query head, the per-head one taking precedence),
+  prefix-LM (causal, plus every key of the sequence's first ``prefix_len``
+  positions), and documents (sequences packed from several documents: causal
+  and both positions in the same document, documents being the runs between
+  consecutive start positions).
 * Query head ``h`` reads KV head ``h // (Hq / Hkv)`` (contiguous grouping).
 * ``lse`` is the natural-log log-sum-exp of the scaled, masked scores. A row
   that sees no key returns ``out = 0`` and ``lse = -inf``.
@@ -28,6 +33,8 @@ import numpy as np
 MASK_NONE = 0
 MASK_CAUSAL = 1
 MASK_SLIDING = 2
+MASK_PREFIX_LM = 3
+MASK_DOCUMENT = 4
 
 
 def _f64(x):
@@ -45,21 +52,37 @@ def _i64(x):
     return np.asarray(x, dtype=np.int64)
 
 
-def visible(kind, q_pos, k_pos, window):
+def document_of(doc_starts, pos):
+    """Index of the document holding each position: the number of document
+    start positions at or before it."""
+    starts = np.sort(np.asarray(doc_starts, dtype=np.int64))
+    return np.searchsorted(starts, np.asarray(pos), side="right")
+
+
+def visible(kind, q_pos, k_pos, window, prefix_len=0, doc_starts=None):
     """Mask modifier: may query position ``q_pos`` see key position ``k_pos``?
 
     Works elementwise on broadcastable integer arrays. Keys beyond the
     sequence are never passed in, so ``none`` is always true here.
+    ``window`` is the sliding window of this (sequence, head); ``prefix_len``
+    the sequence's bidirectional prefix (prefix-LM); ``doc_starts`` the
+    sequence's document start positions (documents).
     """
     q_pos = np.asarray(q_pos)
     k_pos = np.asarray(k_pos)
     if kind == MASK_NONE:
         return np.ones(np.broadcast(q_pos, k_pos).shape, dtype=bool)
     causal = k_pos <= q_pos
-    if kind == MASK_CAUSAL or window is None or window <= 0:
+    if kind == MASK_CAUSAL:
         return causal
     if kind == MASK_SLIDING:
+        if window is None or window <= 0:
+            return causal
         return causal & (q_pos - k_pos < window)
+    if kind == MASK_PREFIX_LM:
+        return causal | (k_pos < prefix_len)
+    if kind == MASK_DOCUMENT:
+        return causal & (document_of(doc_starts, q_pos) == document_of(doc_starts, k_pos))
     raise ValueError(f"unknown mask kind {kind}")
 
 
@@ -82,10 +105,11 @@ def resolve_block_table(cache, table_row, length, block_size):
     return _f64(cache[blocks, :, rows, :])
 
 
-def masked_attention(q, k, v, q_pos, k_pos, scale, kind, window):
+def masked_attention(q, k, v, q_pos, k_pos, scale, kind, window, prefix_len=0, doc_starts=None):
     """Softmax attention of one head.
 
-    q: [nq, d]; k, v: [n, d]; q_pos: [nq]; k_pos: [n].
+    q: [nq, d]; k, v: [n, d]; q_pos: [nq]; k_pos: [n]; the mask arguments are
+    those of ``visible``.
     Returns out [nq, d] and lse [nq] (natural log of the sum of exp of the
     scaled visible scores).
     """
@@ -99,7 +123,8 @@ def masked_attention(q, k, v, q_pos, k_pos, scale, kind, window):
     if k.shape[0] == 0 or nq == 0:
         return out, lse
     s = scale * (q @ k.T)  # [nq, n]
-    vis = visible(kind, np.asarray(q_pos)[:, None], np.asarray(k_pos)[None, :], window)
+    vis = visible(kind, np.asarray(q_pos)[:, None], np.asarray(k_pos)[None, :], window,
+                  prefix_len, doc_starts)
     s = np.where(vis, s, -np.inf)
     any_vis = vis.any(axis=1)
     m = np.where(any_vis, s.max(axis=1), 0.0)
@@ -111,18 +136,32 @@ def masked_attention(q, k, v, q_pos, k_pos, scale, kind, window):
     return out, lse
 
 
-def _window_of(b, window, window_per_seq):
-    if window_per_seq is not None:
-        return int(_i64(window_per_seq)[b])
-    return int(window) if window is not None else 0
+def _mask_of(b, h, window, window_per_seq, window_per_head, prefix_len, doc_offsets,
+             doc_starts):
+    """(window, prefix_len, doc_starts) of sequence b, query head h."""
+    if window_per_head is not None:
+        w = int(_i64(window_per_head)[h])
+    elif window_per_seq is not None:
+        w = int(_i64(window_per_seq)[b])
+    else:
+        w = int(window) if window is not None else 0
+    P = int(_i64(prefix_len)[b]) if prefix_len is not None else 0
+    starts = None
+    if doc_offsets is not None:
+        off = _i64(doc_offsets)
+        starts = _i64(doc_starts)[off[b]:off[b + 1]]
+    return w, P, starts
 
 
 def paged_decode_rows(q, k_cache, v_cache, block_tables, seq_lens, scale, kind,
-                      window=0, window_per_seq=None, rows=None):
+                      window=0, window_per_seq=None, rows=None, window_per_head=None,
+                      prefix_len=None, doc_offsets=None, doc_starts=None):
     """Decode attention for selected (b, h) pairs (all pairs when rows is None).
 
     One query token per sequence at position ``seq_lens[b] - 1`` (the token
     just appended) attends to the sequence's first ``seq_lens[b]`` keys.
+    Mask arguments: ``window_per_head`` [Hq], ``prefix_len`` [B], and the
+    documents of sequence b at ``doc_starts[doc_offsets[b]:doc_offsets[b+1]]``.
     Returns dict (b, h) -> (out [d], lse).
     """
     q = _f64(q)
@@ -143,19 +182,21 @@ def paged_decode_rows(q, k_cache, v_cache, block_tables, seq_lens, scale, kind,
                            resolve_block_table(v_cache, tables[b], L, bs))
         K, V = cache_kv[b]
         kvh = h // g
+        w, P, starts = _mask_of(b, h, window, window_per_seq, window_per_head, prefix_len,
+                                doc_offsets, doc_starts)
         o, l = masked_attention(q[b, h][None, :], K[:, kvh, :], V[:, kvh, :],
-                                np.array([L - 1]), np.arange(L), scale, kind,
-                                _window_of(b, window, window_per_seq))
+                                np.array([L - 1]), np.arange(L), scale, kind, w, P, starts)
         res[(b, h)] = (o[0], l[0])
     return res
 
 
 def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale, kind,
-                 window=0, window_per_seq=None):
-    """Full decode: out [B, Hq, d] float64, lse [B, Hq] float64."""
+                 window=0, window_per_seq=None, **mask):
+    """Full decode: out [B, Hq, d] float64, lse [B, Hq] float64. ``mask`` takes
+    the further mask arguments of ``paged_decode_rows``."""
     B, Hq, d = q.shape
     res = paged_decode_rows(q, k_cache, v_cache, block_tables, seq_lens, scale, kind,
-                            window, window_per_seq)
+                            window, window_per_seq, **mask)
     out = np.zeros((B, Hq, d))
     lse = np.zeros((B, Hq))
     for (b, h), (o, l) in res.items():
@@ -165,7 +206,9 @@ def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale, kind,
 
 
 def paged_prefill_rows(q, k_new, v_new, k_cache, v_cache, block_tables, ctx_lens, q_lens,
-                       scale, kind, window=0, window_per_seq=None, rows=None):
+                       scale, kind, window=0, window_per_seq=None, rows=None,
+                       window_per_head=None, prefix_len=None, doc_offsets=None,
+                       doc_starts=None):
     """Chunked prefill for selected (b, h, i) rows (all rows when rows is None).
 
     Sequence b has ``ctx_lens[b]`` tokens already in the paged cache, followed
@@ -201,18 +244,21 @@ def paged_prefill_rows(q, k_new, v_new, k_cache, v_cache, block_tables, ctx_lens
         K, V = kv_of[b]
         kvh = h // g
         n = C + Q
+        w, P, dst = _mask_of(b, h, window, window_per_seq, window_per_head, prefix_len,
+                             doc_offsets, doc_starts)
         o, l = masked_attention(q[starts[b] + i, h][None, :], K[:, kvh, :], V[:, kvh, :],
-                                np.array([C + i]), np.arange(n), scale, kind,
-                                _window_of(b, window, window_per_seq))
+                                np.array([C + i]), np.arange(n), scale, kind, w, P, dst)
         res[(b, h, i)] = (o[0], l[0])
     return res
 
 
 def paged_prefill(q, k_new, v_new, k_cache, v_cache, block_tables, ctx_lens, q_lens,
-                  scale, kind, window=0, window_per_seq=None):
+                  scale, kind, window=0, window_per_seq=None, window_per_head=None,
+                  prefix_len=None, doc_offsets=None, doc_starts=None):
     """Full chunked prefill: out [sum Q, Hq, d], lse [sum Q, Hq] (float64).
 
-    Computed head by head as one matrix of queries per sequence.
+    Computed head by head as one matrix of queries per sequence; mask
+    arguments as in ``paged_prefill_rows``.
     """
     q = _f64(q)
     ctx = _i64(ctx_lens)
@@ -231,10 +277,11 @@ def paged_prefill(q, k_new, v_new, k_cache, v_cache, block_tables, ctx_lens, q_l
         vctx = resolve_block_table(v_cache, tables[b], C, bs)
         K = np.concatenate([kctx, _f64(k_new[start:start + Q])], axis=0)
         V = np.concatenate([vctx, _f64(v_new[start:start + Q])], axis=0)
-        w = _window_of(b, window, window_per_seq)
         for h in range(Hq):
+            w, P, dst = _mask_of(b, h, window, window_per_seq, window_per_head, prefix_len,
+                                 doc_offsets, doc_starts)
             o, l = masked_attention(q[start:start + Q, h], K[:, h // g], V[:, h // g],
-                                    C + np.arange(Q), np.arange(C + Q), scale, kind, w)
+                                    C + np.arange(Q), np.arange(C + Q), scale, kind, w, P, dst)
             out[start:start + Q, h] = o
             lse[start:start + Q, h] = l
         start += Q

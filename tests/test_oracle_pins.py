@@ -28,18 +28,30 @@ pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
 
 # ----------------------------------------------------------------- brute force
 
-def brute_visible(kind, qp, kp, w):
+def brute_doc(starts, p):
+    n = 0
+    for st in starts:
+        if st <= p:
+            n += 1
+    return n
+
+
+def brute_visible(kind, qp, kp, w, P=0, starts=()):
     if kind == 0:
+        return True
+    if kind == 3 and kp < P:
         return True
     if kp > qp:
         return False
     if kind == 2 and w > 0 and qp - kp >= w:
         return False
+    if kind == 4 and brute_doc(starts, qp) != brute_doc(starts, kp):
+        return False
     return True
 
 
 def brute_paged_attention(qrow, k_cache, v_cache, table, n_keys, q_pos, kvh, scale, kind, w,
-                          extra_k=(), extra_v=()):
+                          extra_k=(), extra_v=(), P=0, starts=()):
     """Scalar loops over Python lists; keys 0..n_keys-1 come from the paged
     cache, further keys (positions n_keys, n_keys+1, ...) from extra_k/extra_v."""
     bs = len(k_cache[0][0])
@@ -52,7 +64,7 @@ def brute_paged_attention(qrow, k_cache, v_cache, table, n_keys, q_pos, kvh, sca
     vals += list(extra_v)
     scores = []
     for p, k in enumerate(keys):
-        if brute_visible(kind, q_pos, p, w):
+        if brute_visible(kind, q_pos, p, w, P, starts):
             s = 0.0
             for a, b in zip(qrow, k):
                 s += a * b
@@ -153,7 +165,7 @@ def test_rows_api_matches_full():
 
 # ----------------------------------------------------------------- planted mistakes
 
-def _mut_causal_strict(kind, q_pos, k_pos, window):
+def _mut_causal_strict(kind, q_pos, k_pos, window, prefix_len=0, doc_starts=None):
     q_pos, k_pos = np.asarray(q_pos), np.asarray(k_pos)
     if kind == A.MASK_NONE:
         return np.ones(np.broadcast(q_pos, k_pos).shape, dtype=bool)
@@ -163,7 +175,7 @@ def _mut_causal_strict(kind, q_pos, k_pos, window):
     return c
 
 
-def _mut_window_inclusive(kind, q_pos, k_pos, window):
+def _mut_window_inclusive(kind, q_pos, k_pos, window, prefix_len=0, doc_starts=None):
     q_pos, k_pos = np.asarray(q_pos), np.asarray(k_pos)
     if kind == A.MASK_NONE:
         return np.ones(np.broadcast(q_pos, k_pos).shape, dtype=bool)
@@ -419,3 +431,181 @@ def test_copy_blocks_brute_force():
         src = {4: 1, 0: 5}.get(blk, blk)
         assert torch.equal(ek[blk], kc[src]) and torch.equal(ev[blk], vc[src])
     assert torch.equal(kc, torch.arange(6 * 2 * 4 * 3, dtype=torch.float32).view(6, 2, 4, 3))
+
+
+# ----------------------------------------------------------------- further mask_mods
+
+def _docs_csr(per_seq):
+    off = np.concatenate([[0], np.cumsum([len(x) for x in per_seq])]).astype(np.int64)
+    flat = np.concatenate([np.asarray(x, dtype=np.int64) for x in per_seq]) if per_seq else \
+        np.zeros(0, dtype=np.int64)
+    return off, flat
+
+
+MASK_CASES = [
+    # (kind, per-head windows, prefix lens, document starts per sequence)
+    (A.MASK_PREFIX_LM, None, [6, 30], None),
+    (A.MASK_PREFIX_LM, None, [0, 41], None),
+    (A.MASK_DOCUMENT, None, None, [[0, 5, 9], [0, 17, 18, 30]]),
+    (A.MASK_DOCUMENT, None, None, [[3], [0]]),
+    (A.MASK_SLIDING, [3, 0, 7, 1], None, None),
+]
+
+
+@pytest.mark.parametrize("case", MASK_CASES)
+def test_further_masks_decode_match_brute_force(case):
+    kind, wph, plen, docs = case
+    B, Hq, Hkv, d, bs, NB = 2, 4, 2, 8, 4, 40
+    lens = [13, 38]
+    q, kc, vc, tab, lens, scale = tiny_case(31, B, Hq, Hkv, d, bs, NB, lens, kind, 0)
+    off, flat = _docs_csr(docs) if docs else (None, None)
+    out, lse = oracle.paged_decode(q, kc, vc, tab, lens, scale, kind, 0, None,
+                                   window_per_head=wph, prefix_len=plen, doc_offsets=off,
+                                   doc_starts=flat)
+    kl, vl, ql = kc.tolist(), vc.tolist(), q.tolist()
+    g = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            o_ref, l_ref = brute_paged_attention(
+                ql[b][h], kl, vl, tab[b].tolist(), int(lens[b]), int(lens[b]) - 1, h // g, scale,
+                kind, wph[h] if wph else 0, P=plen[b] if plen else 0,
+                starts=docs[b] if docs else ())
+            np.testing.assert_allclose(out[b, h], o_ref, rtol=0, atol=1e-13)
+            assert abs(lse[b, h] - l_ref) < 1e-13
+
+
+@pytest.mark.parametrize("case", MASK_CASES)
+def test_further_masks_prefill_match_brute_force(case):
+    kind, wph, plen, docs = case
+    B, Hq, Hkv, d, bs = 2, 4, 2, 8, 4
+    ctx, ql = [9, 22], [6, 19]
+    gen = torch.Generator().manual_seed(8)
+    q, kc, vc, tab, _, scale = tiny_case(8, B, Hq, Hkv, d, bs, 40,
+                                         [c + n for c, n in zip(ctx, ql)], kind, 0)
+    T = sum(ql)
+    qp = torch.randn(T, Hq, d, generator=gen, dtype=torch.float64)
+    kn = torch.randn(T, Hkv, d, generator=gen, dtype=torch.float64)
+    vn = torch.randn(T, Hkv, d, generator=gen, dtype=torch.float64)
+    off, flat = _docs_csr(docs) if docs else (None, None)
+    out, lse = oracle.paged_prefill(qp, kn, vn, kc, vc, tab, ctx, ql, scale, kind, 0, None,
+                                    window_per_head=wph, prefix_len=plen, doc_offsets=off,
+                                    doc_starts=flat)
+    kl, vl = kc.tolist(), vc.tolist()
+    g = Hq // Hkv
+    start = 0
+    for b in range(B):
+        for i in range(ql[b]):
+            for h in range(Hq):
+                ek = [kn[start + j, h // g].tolist() for j in range(ql[b])]
+                ev = [vn[start + j, h // g].tolist() for j in range(ql[b])]
+                o_ref, l_ref = brute_paged_attention(
+                    qp[start + i, h].tolist(), kl, vl, tab[b].tolist(), ctx[b], ctx[b] + i,
+                    h // g, scale, kind, wph[h] if wph else 0, ek, ev,
+                    P=plen[b] if plen else 0, starts=docs[b] if docs else ())
+                np.testing.assert_allclose(out[start + i, h], o_ref, rtol=0, atol=1e-13)
+                assert abs(lse[start + i, h] - l_ref) < 1e-13
+        start += ql[b]
+
+
+def test_packed_documents_equal_separate_sequences():
+    """A sequence packed from documents, under the document mask, gives for each
+    query exactly causal attention over its own document alone (positions
+    rebased), computed as a separate contiguous sequence."""
+    gen = torch.Generator().manual_seed(4)
+    Hq, Hkv, d = 4, 2, 16
+    starts = [0, 7, 20, 21, 40]
+    n = 52
+    K = torch.randn(n, Hkv, d, generator=gen, dtype=torch.float64)
+    V = torch.randn(n, Hkv, d, generator=gen, dtype=torch.float64)
+    Qm = torch.randn(n, Hq, d, generator=gen, dtype=torch.float64)
+    scale = 0.3
+    # packed: the whole sequence as one chunk with no context (identity layout, bs 4)
+    bs = 4
+    kc = K.view(n // bs, bs, Hkv, d).permute(0, 2, 1, 3).contiguous()
+    vc = V.view(n // bs, bs, Hkv, d).permute(0, 2, 1, 3).contiguous()
+    tab = np.arange(n // bs)[None, :]
+    out, lse = oracle.paged_prefill(Qm, K, V, kc, vc, tab, [0], [n], scale, A.MASK_DOCUMENT,
+                                    doc_offsets=[0, len(starts)], doc_starts=starts)
+    bounds = starts + [n]
+    for s0, s1 in zip(bounds[:-1], bounds[1:]):
+        for h in range(Hq):
+            o_ref, l_ref = A.masked_attention(Qm[s0:s1, h], K[s0:s1, h // 2], V[s0:s1, h // 2],
+                                              np.arange(s1 - s0), np.arange(s1 - s0), scale,
+                                              A.MASK_CAUSAL, 0)
+            np.testing.assert_allclose(out[s0:s1, h], o_ref, rtol=0, atol=1e-13)
+            np.testing.assert_allclose(lse[s0:s1, h], l_ref, rtol=0, atol=1e-13)
+
+
+def test_prefix_lm_limits():
+    """prefix_len 0 is causal; a prefix covering every key is no mask."""
+    q, kc, vc, tab, lens, scale = tiny_case(9, 2, 4, 2, 8, 4, 40, [20, 33], A.MASK_CAUSAL, 0)
+    ctx, ql = [8, 12], [12, 21]
+    gen = torch.Generator().manual_seed(9)
+    qp = torch.randn(33, 4, 8, generator=gen, dtype=torch.float64)
+    kn = torch.randn(33, 2, 8, generator=gen, dtype=torch.float64)
+    vn = torch.randn(33, 2, 8, generator=gen, dtype=torch.float64)
+    causal = oracle.paged_prefill(qp, kn, vn, kc, vc, tab, ctx, ql, scale, A.MASK_CAUSAL)
+    p0 = oracle.paged_prefill(qp, kn, vn, kc, vc, tab, ctx, ql, scale, A.MASK_PREFIX_LM,
+                              prefix_len=[0, 0])
+    none = oracle.paged_prefill(qp, kn, vn, kc, vc, tab, ctx, ql, scale, A.MASK_NONE)
+    full = oracle.paged_prefill(qp, kn, vn, kc, vc, tab, ctx, ql, scale, A.MASK_PREFIX_LM,
+                                prefix_len=[20, 33])
+    for a, b in ((causal, p0), (none, full)):
+        np.testing.assert_array_equal(a[0], b[0])
+        np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_per_head_windows_equal_one_window_per_call():
+    q, kc, vc, tab, lens, scale = tiny_case(12, 3, 4, 2, 8, 4, 60, [5, 30, 47],
+                                            A.MASK_SLIDING, 0)
+    wph = [1, 9, 0, 30]
+    out, lse = oracle.paged_decode(q, kc, vc, tab, lens, scale, A.MASK_SLIDING, 0,
+                                   window_per_head=wph)
+    for h, w in enumerate(wph):
+        o1, l1 = oracle.paged_decode(q, kc, vc, tab, lens, scale, A.MASK_SLIDING, w)
+        np.testing.assert_array_equal(out[:, h], o1[:, h])
+        np.testing.assert_array_equal(lse[:, h], l1[:, h])
+
+
+def _mut_prefix_inclusive(kind, q_pos, k_pos, window, prefix_len=0, doc_starts=None):
+    q_pos, k_pos = np.asarray(q_pos), np.asarray(k_pos)
+    return (k_pos <= q_pos) | (k_pos <= prefix_len)  # planted: prefix one key too long
+
+
+def _mut_doc_start_in_previous(kind, q_pos, k_pos, window, prefix_len=0, doc_starts=None):
+    q_pos, k_pos = np.asarray(q_pos), np.asarray(k_pos)
+    st = np.sort(np.asarray(doc_starts))
+    d = lambda p: np.searchsorted(st, p, side="left")  # planted: a start joins the previous doc
+    return (k_pos <= q_pos) & (d(q_pos) == d(k_pos))
+
+
+@pytest.mark.parametrize("mutation", ["prefix_inclusive", "doc_start_in_previous"])
+def test_planted_mask_mistakes_are_caught(monkeypatch, mutation):
+    kind = A.MASK_PREFIX_LM if mutation == "prefix_inclusive" else A.MASK_DOCUMENT
+    plen, docs = [6, 30], [[0, 5, 9], [0, 17, 18, 30]]
+    q, kc, vc, tab, lens, scale = tiny_case(31, 2, 4, 2, 8, 4, 40, [13, 38], kind, 0)
+    off, flat = _docs_csr(docs)
+    monkeypatch.setattr(A, "visible", _mut_prefix_inclusive if mutation == "prefix_inclusive"
+                        else _mut_doc_start_in_previous)
+    # decode queries see the whole prefix anyway: plant in a prefill
+    ctx, ql = [9, 22], [4, 16]
+    gen = torch.Generator().manual_seed(8)
+    qp = torch.randn(20, 4, 8, generator=gen, dtype=torch.float64)
+    kn = torch.randn(20, 2, 8, generator=gen, dtype=torch.float64)
+    vn = torch.randn(20, 2, 8, generator=gen, dtype=torch.float64)
+    out, lse = A.paged_prefill(qp, kn, vn, kc, vc, tab, ctx, ql, scale, kind, prefix_len=plen,
+                               doc_offsets=off, doc_starts=flat)
+    monkeypatch.undo()
+    kl, vl = kc.tolist(), vc.tolist()
+    worst, start = 0.0, 0
+    for b in range(2):
+        for i in range(ql[b]):
+            for h in range(4):
+                ek = [kn[start + j, h // 2].tolist() for j in range(ql[b])]
+                ev = [vn[start + j, h // 2].tolist() for j in range(ql[b])]
+                o_ref, l_ref = brute_paged_attention(
+                    qp[start + i, h].tolist(), kl, vl, tab[b].tolist(), ctx[b], ctx[b] + i,
+                    h // 2, scale, kind, 0, ek, ev, P=plen[b], starts=docs[b])
+                worst = max(worst, float(np.max(np.abs(out[start + i, h] - o_ref))))
+        start += ql[b]
+    assert worst > 1e-6, f"mutation {mutation} went unnoticed"
