@@ -72,19 +72,44 @@ extern "C" {
 typedef enum { PKV_F32 = 0, PKV_BF16 = 1 } pkv_dtype;
 
 typedef enum {
-  PKV_MASK_NONE = 0,    /* every key of the sequence is visible */
-  PKV_MASK_CAUSAL = 1,  /* key position <= query position */
-  PKV_MASK_SLIDING = 2  /* causal and query - key < window (window keys incl. self) */
+  PKV_MASK_NONE = 0,      /* every key of the sequence is visible */
+  PKV_MASK_CAUSAL = 1,    /* key position <= query position */
+  PKV_MASK_SLIDING = 2,   /* causal and query - key < window (window keys incl. self) */
+  PKV_MASK_PREFIX_LM = 3, /* causal, plus every key below the sequence's prefix_len */
+  PKV_MASK_DOCUMENT = 4   /* causal within documents packed into one sequence */
 } pkv_mask_kind;
 
 /* FlexAttention-style mask modifier, as data (a C ABI cannot take a callable).
- * window <= 0 with PKV_MASK_SLIDING means causal only. window_per_seq, when
- * not NULL, is a device int32 [batch] array that overrides `window` per
- * sequence (same <= 0 rule). */
+ * "Paged Attention Meets FlexAttention" (abstract) applies FlexAttention mask
+ * modifiers inside the paged kernel; the kinds here are the ones whose
+ * visible keys, for a query at position q, form one interval [lo(q), hi(q))
+ * with both ends non-decreasing in q, so whole tiles outside it are skipped
+ * and only boundary tiles are masked element by element.
+ *   window           PKV_MASK_SLIDING: keys q-window+1 .. q are visible;
+ *                    window <= 0 means causal only.
+ *   window_per_seq   device int32 [batch] or NULL: overrides `window` per
+ *                    sequence (same <= 0 rule).
+ *   window_per_head  device int32 [num_q_heads] or NULL: overrides both per
+ *                    query head (same rule). The decode kernels read the union
+ *                    of the heads' ranges and mask each head's own.
+ *   prefix_len       PKV_MASK_PREFIX_LM: device int32 [batch]; keys below
+ *                    prefix_len[b] are visible to every query of sequence b
+ *                    (a bidirectional prefix), the rest causally.
+ *   doc_offsets      PKV_MASK_DOCUMENT: device int32 [batch + 1]; sequence b's
+ *   doc_starts       document start positions are doc_starts[doc_offsets[b]
+ *                    .. doc_offsets[b+1]-1], ascending. A document runs from
+ *                    its start to the next start; positions before the first
+ *                    start form a document of their own. A query sees the keys
+ *                    of its own document up to itself.
+ * Pointers a kind does not use are ignored. */
 typedef struct {
   int32_t kind;
   int32_t window;
   const int32_t* window_per_seq;
+  const int32_t* window_per_head;
+  const int32_t* prefix_len;
+  const int32_t* doc_offsets;
+  const int32_t* doc_starts;
 } pkv_mask_mod;
 
 /* Shape of one K (or V) pool. */

@@ -20,6 +20,7 @@ from .ops import (  # noqa: F401
     causal,
     decode_workspace,
     decode_workspace_size,
+    document,
     no_mask,
     paged_attention_decode,
     paged_attention_decode_shared_prefix,
@@ -27,6 +28,7 @@ from .ops import (  # noqa: F401
     paged_kv_append,
     paged_kv_copy_blocks,
     paged_kv_gather,
+    prefix_lm,
     read_dbg,
     shared_prefix_workspace,
     shared_prefix_workspace_size,

@@ -30,6 +30,8 @@ PKV_BF16 = 1
 PKV_MASK_NONE = 0
 PKV_MASK_CAUSAL = 1
 PKV_MASK_SLIDING = 2
+PKV_MASK_PREFIX_LM = 3
+PKV_MASK_DOCUMENT = 4
 
 # every symbol the header declares; the CPU test checks that all are exported
 EXPORTS = (
@@ -51,7 +53,9 @@ EXPORTS = (
 
 class MaskModC(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("window", ctypes.c_int32),
-                ("window_per_seq", ctypes.c_void_p)]
+                ("window_per_seq", ctypes.c_void_p), ("window_per_head", ctypes.c_void_p),
+                ("prefix_len", ctypes.c_void_p), ("doc_offsets", ctypes.c_void_p),
+                ("doc_starts", ctypes.c_void_p)]
 
 
 class CacheDescC(ctypes.Structure):

@@ -110,8 +110,12 @@ int check_cache(const pkv_cache_desc& c, const char* fn) {
 }
 
 int check_mask(const pkv_mask_mod& m, const char* fn) {
-  if (m.kind != PKV_MASK_NONE && m.kind != PKV_MASK_CAUSAL && m.kind != PKV_MASK_SLIDING)
+  if (m.kind < PKV_MASK_NONE || m.kind > PKV_MASK_DOCUMENT)
     return fail(PKV_ERR_INVALID_ARG, "%s: unknown mask kind %d", fn, m.kind);
+  if (m.kind == PKV_MASK_PREFIX_LM && !m.prefix_len)
+    return fail(PKV_ERR_INVALID_ARG, "%s: prefix-LM mask needs prefix_len", fn);
+  if (m.kind == PKV_MASK_DOCUMENT && (!m.doc_offsets || !m.doc_starts))
+    return fail(PKV_ERR_INVALID_ARG, "%s: document mask needs doc_offsets and doc_starts", fn);
   return PKV_OK;
 }
 

@@ -743,8 +743,8 @@ PKV_API int paged_attention_decode_shared_prefix(
     return fail(PKV_ERR_UNSUPPORTED, "%s: bf16 pools with head_dim 128 only", fn);
   if (cache.block_size < 8)
     return fail(PKV_ERR_UNSUPPORTED, "%s: block_size must be >= 8", fn);
-  if (mask.kind == PKV_MASK_SLIDING)
-    return fail(PKV_ERR_UNSUPPORTED, "%s: mask must be none or causal", fn);
+  if (mask.kind == PKV_MASK_SLIDING || mask.kind == PKV_MASK_DOCUMENT)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: mask must be none, causal or prefix-LM", fn);
   if (batch < 0 || max_blocks_per_seq <= 0)
     return fail(PKV_ERR_INVALID_ARG, "%s: bad batch or max_blocks_per_seq", fn);
   if (num_q_heads <= 0 || num_q_heads % cache.num_kv_heads)

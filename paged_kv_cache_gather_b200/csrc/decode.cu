@@ -53,9 +53,7 @@ struct DecodeParams {
   int32_t bs_shift;    // log2(block_size)
   int32_t num_blocks;
   float scale_log2;    // scale * log2(e)
-  int32_t mask_kind;
-  int32_t window;
-  const int32_t* window_per_seq;
+  pkv_mask_mod mask;
   __nv_bfloat16* out;
   float* lse;
   float* ws_o;         // [2 * workers, group, D] partial outputs (normalised)
@@ -81,7 +79,7 @@ __device__ __forceinline__ SeqSpan seq_span(const DecodeParams& p, int b) {
     flag_error(p.dbg, PKV_DBG_LENGTH);
     L = cap;
   }
-  decode_key_range(p.mask_kind, p.window, p.window_per_seq, b, L, s.lo, s.hi);
+  decode_key_range(p.mask, p.num_q_heads, b, L, s.lo, s.hi);
   s.t0 = s.lo / kTile;
   s.n = s.hi > s.lo ? (s.hi + kTile - 1) / kTile - s.t0 : 0;
   return s;
@@ -182,7 +180,9 @@ struct Cfg {
   static constexpr int kStageBytes = 2 * kTileBytes;      // K then V
 };
 
-template <int D, int NSTAGE, int WPC>
+// PH: per-head sliding windows (each head column masks keys below its own
+// start); the instance without them carries none of that code.
+template <int D, int NSTAGE, int WPC, bool PH>
 __global__ void __launch_bounds__(WPC * 32, 1)
     decode_bf16_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
@@ -302,6 +302,10 @@ __global__ void __launch_bounds__(WPC * 32, 1)
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   int piece = 0;  // 0 for the worker's first piece, 1 afterwards
   int64_t piece_start = start;
+  // per-head windows: the segment spans the union of the heads' ranges and
+  // each of this lane's two head columns masks keys below its own start
+  constexpr bool per_head = PH;
+  int lo_h0 = 0, lo_h1 = 0;
 
   for (int64_t k = 0; k < ntiles; ++k) {
     // producer: refill the stage consumed in the previous iteration
@@ -325,6 +329,12 @@ __global__ void __launch_bounds__(WPC * 32, 1)
         } else {
           qf[kk][0] = qf[kk][1] = 0u;
         }
+      }
+      if (per_head) {
+        const int L = cur.s.hi;
+        const int hb = cur.kvh * p.group + 2 * c4;
+        lo_h0 = 2 * c4 < p.group ? mask_lo(p.mask, cur.b, hb, L - 1) : 0;
+        lo_h1 = 2 * c4 + 1 < p.group ? mask_lo(p.mask, cur.b, hb + 1, L - 1) : 0;
       }
 #pragma unroll
       for (int mt = 0; mt < D / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
@@ -382,19 +392,33 @@ __global__ void __launch_bounds__(WPC * 32, 1)
       if (p0 < cur.s.lo || p0 >= cur.s.hi) x[0] = x[1] = -INFINITY;
       if (p1 < cur.s.lo || p1 >= cur.s.hi) x[2] = x[3] = -INFINITY;
     }
+    if (per_head) {
+      const int p0 = tok0 + g4, p1 = p0 + 8;
+      if (p0 < lo_h0) x[0] = -INFINITY;
+      if (p0 < lo_h1) x[1] = -INFINITY;
+      if (p1 < lo_h0) x[2] = -INFINITY;
+      if (p1 < lo_h1) x[3] = -INFINITY;
+    }
     float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
     }
-    // every tile of a piece holds a visible key, so the new maxima are finite
+    // every tile of a piece holds a key visible to all heads of the group, so
+    // the new maxima are finite; with per-head windows a head may have seen
+    // none yet (maximum -inf), and 0 stands in as the reference then
     const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-    const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);
+    float r0 = n0, r1 = n1;
+    if (per_head) {
+      r0 = n0 == -INFINITY ? 0.f : n0;
+      r1 = n1 == -INFINITY ? 0.f : n1;
+    }
+    const float al0 = fast_exp2(m0 - r0), al1 = fast_exp2(m1 - r1);
     m0 = n0;
     m1 = n1;
-    const float p00 = fast_exp2(x[0] - n0), p01 = fast_exp2(x[1] - n1);
-    const float p10 = fast_exp2(x[2] - n0), p11 = fast_exp2(x[3] - n1);
+    const float p00 = fast_exp2(x[0] - r0), p01 = fast_exp2(x[1] - r1);
+    const float p10 = fast_exp2(x[2] - r0), p11 = fast_exp2(x[3] - r1);
     l0 = l0 * al0 + p00 + p10;
     l1 = l1 * al1 + p01 + p11;
     if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
@@ -431,8 +455,10 @@ __global__ void __launch_bounds__(WPC * 32, 1)
         s0 += __shfl_xor_sync(0xffffffffu, s0, off);
         s1 += __shfl_xor_sync(0xffffffffu, s1, off);
       }
-      const float inv0 = 1.f / s0, inv1 = 1.f / s1;
-      const float lse0 = m0 * kLn2 + logf(s0), lse1 = m1 * kLn2 + logf(s1);
+      // a head that saw no key in this piece (per-head windows) gives 0, -inf
+      const float inv0 = s0 > 0.f ? 1.f / s0 : 0.f, inv1 = s1 > 0.f ? 1.f / s1 : 0.f;
+      const float lse0 = s0 > 0.f ? m0 * kLn2 + logf(s0) : -INFINITY;
+      const float lse1 = s1 > 0.f ? m1 * kLn2 + logf(s1) : -INFINITY;
       const int h0 = 2 * c4, h1 = h0 + 1;
       const bool whole = (piece_start == cur.seg_first) && (cur.t + 1 == seg_end);
       if (whole) {
@@ -593,8 +619,8 @@ __global__ void __launch_bounds__(128) decode_f32_kernel(
     const float* __restrict__ q, const float* __restrict__ kc, const float* __restrict__ vc,
     const int32_t* __restrict__ tables, int32_t max_blocks, const int32_t* __restrict__ seq_lens,
     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t bs_shift,
-    int32_t num_blocks, float scale, int32_t mask_kind, int32_t window,
-    const int32_t* window_per_seq, float* __restrict__ out, float* __restrict__ lse, int32_t* dbg) {
+    int32_t num_blocks, float scale, pkv_mask_mod mask, float* __restrict__ out,
+    float* __restrict__ lse, int32_t* dbg) {
   constexpr int NT = 128;
   __shared__ float qs[256];
   __shared__ float ps[NT];
@@ -610,7 +636,8 @@ __global__ void __launch_bounds__(128) decode_f32_kernel(
     L = max_blocks << bs_shift;
   }
   int lo, hi;
-  decode_key_range(mask_kind, window, window_per_seq, b, L, lo, hi);
+  hi = L;
+  lo = L > 0 ? mask_lo(mask, b, h, L - 1) : 0;
   for (int d = tid; d < head_dim; d += NT) qs[d] = q[((int64_t)b * num_q_heads + h) * head_dim + d];
   __syncthreads();
   float m = -INFINITY, l = 0.f;
@@ -682,7 +709,7 @@ __global__ void __launch_bounds__(128) decode_f32_kernel(
 
 namespace {
 
-template <int D, int NSTAGE, int WPC>
+template <int D, int NSTAGE, int WPC, bool PH>
 int launch_bf16_impl(const DecodeArgs& a) {
   using Cf = Cfg<D>;
   const int sms = device_sm_count();
@@ -693,7 +720,7 @@ int launch_bf16_impl(const DecodeArgs& a) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(decode_bf16_kernel<D, NSTAGE, WPC>,
+    if (cudaFuncSetAttribute(decode_bf16_kernel<D, NSTAGE, WPC, PH>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return check_launch("paged_attention_decode: smem attribute");
     attr_set[dev] = true;
@@ -718,9 +745,7 @@ int launch_bf16_impl(const DecodeArgs& a) {
   p.bs_shift = log2_int(a.cache.block_size);
   p.num_blocks = a.cache.num_blocks;
   p.scale_log2 = a.scale * kLog2e;
-  p.mask_kind = a.mask.kind;
-  p.window = a.mask.window;
-  p.window_per_seq = a.mask.window_per_seq;
+  p.mask = a.mask;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.lse = a.lse;
   const size_t o_bytes = (size_t)2 * workers * g * D * 4;
@@ -731,7 +756,7 @@ int launch_bf16_impl(const DecodeArgs& a) {
   p.workers = workers;
   p.dbg = a.dbg;
 
-  decode_bf16_kernel<D, NSTAGE, WPC><<<sms, WPC * 32, smem, a.stream>>>(kmap, vmap, p);
+  decode_bf16_kernel<D, NSTAGE, WPC, PH><<<sms, WPC * 32, smem, a.stream>>>(kmap, vmap, p);
   if (int st = check_launch("paged_attention_decode")) return st;
   const int64_t items = (int64_t)a.batch * a.cache.num_kv_heads * g;
   cudaLaunchConfig_t cfg = {};
@@ -764,11 +789,13 @@ int decode_warps_per_cta() {
 template <int D>
 int launch_bf16(const DecodeArgs& a) {
   // 192 KB of ring per CTA for head_dim 128 (8 KB stages), 160-192 KB for 64
+  if (a.mask.kind == PKV_MASK_SLIDING && a.mask.window_per_head)
+    return launch_bf16_impl<D, (D == 128 ? 2 : 4), 12, true>(a);
   switch (decode_warps_per_cta()) {
-    case 6: return launch_bf16_impl<D, (D == 128 ? 4 : 8), 6>(a);
-    case 8: return launch_bf16_impl<D, (D == 128 ? 3 : 6), 8>(a);
-    case 4: return launch_bf16_impl<D, (D == 128 ? 6 : 10), 4>(a);
-    default: return launch_bf16_impl<D, (D == 128 ? 2 : 4), 12>(a);
+    case 6: return launch_bf16_impl<D, (D == 128 ? 4 : 8), 6, false>(a);
+    case 8: return launch_bf16_impl<D, (D == 128 ? 3 : 6), 8, false>(a);
+    case 4: return launch_bf16_impl<D, (D == 128 ? 6 : 10), 4, false>(a);
+    default: return launch_bf16_impl<D, (D == 128 ? 2 : 4), 12, false>(a);
   }
 }
 
@@ -794,7 +821,7 @@ int launch_decode(const DecodeArgs& a) {
         static_cast<const float*>(a.q), static_cast<const float*>(a.k_cache),
         static_cast<const float*>(a.v_cache), a.tables, a.max_blocks, a.seq_lens, a.num_q_heads,
         a.cache.num_kv_heads, a.cache.head_dim, log2_int(a.cache.block_size), a.cache.num_blocks,
-        a.scale, a.mask.kind, a.mask.window, a.mask.window_per_seq, static_cast<float*>(a.out),
+        a.scale, a.mask, static_cast<float*>(a.out),
         a.lse, a.dbg);
     return check_launch("paged_attention_decode (fp32)");
   }

@@ -204,15 +204,65 @@ __device__ __forceinline__ void flag_error(int32_t* dbg, int32_t bit) {
   if (dbg) atomicOr(dbg, bit);
 }
 
-// Visible key range [lo, hi) of a decode query at position L-1 under a mask.
-__device__ __forceinline__ void decode_key_range(int32_t kind, int32_t window,
-                                                 const int32_t* window_per_seq, int b, int L,
-                                                 int& lo, int& hi) {
+// ---- mask modifiers: the visible keys of a query at position q form one
+// interval [mask_lo, mask_hi), both ends non-decreasing in q.
+
+// Sliding window of (sequence b, query head h): per head, else per sequence,
+// else the scalar; <= 0 means no window.
+__device__ __forceinline__ int mask_window(const pkv_mask_mod& m, int b, int h) {
+  if (m.window_per_head) return __ldg(m.window_per_head + h);
+  if (m.window_per_seq) return __ldg(m.window_per_seq + b);
+  return m.window;
+}
+
+// Start of the document of sequence b that holds position q: the last listed
+// start <= q (binary search over the ascending starts), or 0 if none.
+__device__ __forceinline__ int mask_doc_start(const pkv_mask_mod& m, int b, int q) {
+  int lo = __ldg(m.doc_offsets + b), hi = __ldg(m.doc_offsets + b + 1);
+  int start = 0;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    const int v = __ldg(m.doc_starts + mid);
+    if (v <= q) {
+      start = v;
+      lo = mid + 1;
+    } else {
+      hi = mid;
+    }
+  }
+  return start;
+}
+
+// First key visible to the query at position q (sequence b, query head h).
+__device__ __forceinline__ int mask_lo(const pkv_mask_mod& m, int b, int h, int q) {
+  if (m.kind == PKV_MASK_SLIDING) {
+    const int w = mask_window(m, b, h);
+    return w > 0 ? max(0, q - w + 1) : 0;
+  }
+  if (m.kind == PKV_MASK_DOCUMENT) return mask_doc_start(m, b, q);
+  return 0;
+}
+
+// One past the last key visible to the query at position q, of n keys.
+__device__ __forceinline__ int mask_hi(const pkv_mask_mod& m, int b, int q, int n) {
+  if (m.kind == PKV_MASK_NONE) return n;
+  int hi = q + 1;
+  if (m.kind == PKV_MASK_PREFIX_LM) hi = max(hi, __ldg(m.prefix_len + b));
+  return min(hi, n);
+}
+
+// Keys a decode query (position L-1) of sequence b reads: [lo, hi). With
+// per-head windows this is the union over the sequence's num_q_heads heads.
+__device__ __forceinline__ void decode_key_range(const pkv_mask_mod& m, int num_q_heads, int b,
+                                                 int L, int& lo, int& hi) {
   hi = L;
   lo = 0;
-  if (kind == PKV_MASK_SLIDING) {
-    int w = window_per_seq ? window_per_seq[b] : window;
-    if (w > 0 && L > w) lo = L - w;
+  if (L <= 0) return;
+  if (m.kind == PKV_MASK_SLIDING && m.window_per_head) {
+    lo = L - 1;
+    for (int h = 0; h < num_q_heads; ++h) lo = min(lo, mask_lo(m, b, h, L - 1));
+  } else {
+    lo = mask_lo(m, b, 0, L - 1);
   }
 }
 

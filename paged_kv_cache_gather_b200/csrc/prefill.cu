@@ -71,9 +71,7 @@ struct PrefillParams {
   int32_t num_blocks;
   int32_t pool_rows;    // num_blocks * Hkv * block_size (first out-of-bounds row)
   float scale_log2;
-  int32_t mask_kind;
-  int32_t window;
-  const int32_t* window_per_seq;
+  pkv_mask_mod mask;
   __nv_bfloat16* out;
   float* lse;
   int32_t* dbg;
@@ -112,14 +110,8 @@ struct Unit {
   int C, Q, qoff;
   int ctx_lo, n_ctx;   // context tiles [ctx_lo, ctx_lo + n_ctx)
   int ch_lo, n_ch;     // chunk tiles   [ch_lo, ch_lo + n_ch)
-  int window;          // <= 0: no window
   __device__ int n() const { return n_ctx + n_ch; }
 };
-
-__device__ __forceinline__ int window_of(const PrefillParams& p, int b) {
-  if (p.mask_kind != PKV_MASK_SLIDING) return 0;
-  return p.window_per_seq ? p.window_per_seq[b] : p.window;
-}
 
 __device__ __forceinline__ Unit unit_of(const PrefillParams& p, const int32_t* qoff, int max_qt,
                                         int64_t u) {
@@ -144,15 +136,18 @@ __device__ __forceinline__ Unit unit_of(const PrefillParams& p, const int32_t* q
     C = cap;
   }
   x.C = C;
-  x.window = window_of(p, x.b);
-  const int qmin = C + x.qt * kM;             // position of the tile's first row
+  const int qmin = C + x.qt * kM;                        // position of the tile's first row
+  const int qlast = min(qmin + kM - 1, C + x.Q - 1);     // and of its last real row
   const int ctx_tiles = (C + kN - 1) / kN;
-  const int q_tiles = (x.Q + kN - 1) / kN;
-  int lo_key = 0;                              // lowest key any row of the tile can see
-  if (x.window > 0) lo_key = max(0, qmin - x.window + 1);
+  // keys any row of the tile can see: [lowest start over the unit's heads at
+  // its first row, end at its last row) (both ends grow with the position)
+  const int h0 = x.kvh * p.group + x.hp * (p.two_heads ? 2 : 1);
+  int lo_key = mask_lo(p.mask, x.b, h0, qmin);
+  if (p.two_heads) lo_key = min(lo_key, mask_lo(p.mask, x.b, h0 + 1, qmin));
+  const int hi_key = mask_hi(p.mask, x.b, qlast, C + x.Q);
   x.ctx_lo = min(lo_key / kN, ctx_tiles);
   x.n_ctx = ctx_tiles - x.ctx_lo;
-  const int ch_hi = (p.mask_kind == PKV_MASK_NONE) ? q_tiles - 1 : min(x.qt, q_tiles - 1);
+  const int ch_hi = hi_key > C ? (hi_key - 1 - C) / kN : -1;
   x.ch_lo = (lo_key > C) ? (lo_key - C) / kN : 0;
   x.n_ch = max(0, ch_hi - x.ch_lo + 1);
   return x;
@@ -534,6 +529,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i_row = x.qt * kM + row;      // query index within the chunk
       const int qpos = x.C + i_row;
       const int qmin = x.C + x.qt * kM, qmax = qmin + kM - 1;
+      // this row's visible keys [row_lo, row_hi); every row of the tile sees
+      // [lo_max, hi_min) (warp-uniform: decides which tiles need no mask)
+      const int h_own = x.kvh * p.group + x.hp * (p.two_heads ? 2 : 1) + hsel;
+      const int n_keys = x.C + x.Q;
+      const int row_lo = mask_lo(p.mask, x.b, h_own, qpos);
+      const int row_hi = mask_hi(p.mask, x.b, qpos, n_keys);
+      const int lo_max = mask_lo(p.mask, x.b, h_own, qmax);
+      const int hi_min = mask_hi(p.mask, x.b, qmin, n_keys);
       float m = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < n; ++j, ++s_cnt) {
@@ -542,10 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ctx;
         int idx, kp0;
         tile_of(x, j, ctx, idx, kp0);
-        const int key_end = ctx ? x.C : x.C + x.Q;
-        bool full = kp0 + kN <= key_end;
-        if (p.mask_kind != PKV_MASK_NONE) full = full && (kp0 + kN - 1 <= qmin);
-        if (x.window > 0) full = full && (qmax - kp0 < x.window);
+        const int key_end = ctx ? x.C : n_keys;
+        const bool full = kp0 + kN <= min(key_end, hi_min) && kp0 >= lo_max;
         // pass 1: the whole S row of this thread in one tensor-memory round trip
         float mx;
         {
@@ -556,9 +557,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!full) {
             // the visible keys of a row form one interval of columns [vlo, vhi);
             // masked scores become -inf in tensor memory, so pass 2 needs no mask
-            int vhi = min(kN, key_end - kp0), vlo = 0;
-            if (p.mask_kind != PKV_MASK_NONE) vhi = min(vhi, qpos - kp0 + 1);
-            if (x.window > 0) vlo = max(0, qpos - x.window + 1 - kp0);
+            const int vhi = min(kN, min(key_end, row_hi) - kp0);
+            const int vlo = max(0, row_lo - kp0);
             const uint32_t span = (uint32_t)max(vhi - vlo, 0);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -719,9 +719,7 @@ int launch_prefill(const PrefillArgs& a) {
   p.pool_rows = (int32_t)pool_rows;
   const float scale = a.scale > 0.f ? a.scale : 1.f / sqrtf((float)kD);
   p.scale_log2 = scale * kLog2e;
-  p.mask_kind = a.mask.kind;
-  p.window = a.mask.window;
-  p.window_per_seq = a.mask.window_per_seq;
+  p.mask = a.mask;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.lse = a.lse;
   p.dbg = a.dbg;

@@ -34,6 +34,8 @@ import torch
 MASK_NONE = 0
 MASK_CAUSAL = 1
 MASK_SLIDING = 2
+MASK_PREFIX_LM = 3
+MASK_DOCUMENT = 4
 
 SEED_BASE = 1234
 
@@ -423,3 +425,37 @@ def config5(batch=4, ctx=30720, chunk=2048, num_blocks=16384, seed=None, peaky=F
                              head_dim=128, block_size=16, num_blocks=num_blocks,
                              seed=seed if seed is not None else seed_for(5),
                              mask_kind=MASK_CAUSAL, peaky=peaky)
+
+
+# --------------------------------------------------------------------------- mask data
+
+def document_starts(lens, seed, mean_doc=200, first_at_zero=True):
+    """Seeded document boundaries for packed sequences: for sequence b, start
+    positions in [0, lens[b]) with gaps drawn from an exponential of mean
+    ``mean_doc`` (at least 1). Returns (doc_offsets int32 [B+1], doc_starts
+    int32), the CSR form the mask takes."""
+    rng = np.random.default_rng(seed)
+    per = []
+    for L in lens:
+        st = [0] if first_at_zero else []
+        p = 0 if first_at_zero else int(rng.integers(1, max(2, mean_doc)))
+        if not first_at_zero and p < L:
+            st.append(p)
+        while True:
+            p += max(1, int(rng.exponential(mean_doc)))
+            if p >= L:
+                break
+            st.append(p)
+        per.append(st)
+    off = np.concatenate([[0], np.cumsum([len(x) for x in per])]).astype(np.int32)
+    flat = np.array([x for st in per for x in st], dtype=np.int32)
+    return torch.from_numpy(off), torch.from_numpy(flat)
+
+
+def with_mask(case, kind, **tensors):
+    """Set a case's mask kind and its further mask tensors (window_per_head,
+    prefix_len, doc_offsets, doc_starts; CPU int32)."""
+    case.mask_kind = kind
+    case.extra["mask"] = {k: v for k, v in tensors.items() if v is not None}
+    case.name += f"_mask{kind}"
+    return case

@@ -22,27 +22,50 @@ _DTYPES = {torch.float32: L.PKV_F32, torch.bfloat16: L.PKV_BF16}
 class MaskMod:
     """FlexAttention-style mask modifier as data.
 
-    kind: ``MaskMod.NONE``, ``CAUSAL`` or ``SLIDING``. ``window`` (sliding only)
-    keeps keys with ``q_pos - k_pos < window``; ``<= 0`` means causal only.
-    ``window_per_seq`` (int32 CUDA tensor [batch]) overrides ``window``.
+    kind: ``MaskMod.NONE``, ``CAUSAL``, ``SLIDING``, ``PREFIX_LM`` or
+    ``DOCUMENT``. ``window`` (sliding) keeps keys with ``q_pos - k_pos <
+    window``; ``<= 0`` means causal only. ``window_per_seq`` (int32 [batch])
+    and ``window_per_head`` (int32 [num_q_heads]) override it, per head first.
+    ``prefix_len`` (int32 [batch], prefix-LM): keys below it are visible to
+    every query. ``doc_offsets`` (int32 [batch + 1]) and ``doc_starts``
+    (int32, ascending per sequence): document start positions of sequence b
+    are ``doc_starts[doc_offsets[b]:doc_offsets[b + 1]]``. All tensors live
+    on the cache's device.
     """
 
     kind: int = L.PKV_MASK_NONE
     window: int = 0
     window_per_seq: Optional[torch.Tensor] = None
+    window_per_head: Optional[torch.Tensor] = None
+    prefix_len: Optional[torch.Tensor] = None
+    doc_offsets: Optional[torch.Tensor] = None
+    doc_starts: Optional[torch.Tensor] = None
 
     NONE = L.PKV_MASK_NONE
     CAUSAL = L.PKV_MASK_CAUSAL
     SLIDING = L.PKV_MASK_SLIDING
+    PREFIX_LM = L.PKV_MASK_PREFIX_LM
+    DOCUMENT = L.PKV_MASK_DOCUMENT
 
-    def to_c(self, batch, device):
-        wps = None
-        if self.window_per_seq is not None:
-            w = self.window_per_seq
-            _check(w.dtype == torch.int32 and w.device == device and w.is_contiguous()
-                   and w.numel() >= batch, "window_per_seq must be int32 [batch] on the device")
-            wps = w.data_ptr()
-        return L.MaskModC(int(self.kind), int(self.window), wps)
+    def to_c(self, batch, device, num_q_heads=None):
+        def arr(t, n, name):
+            if t is None:
+                return None
+            _check(t.dtype == torch.int32 and t.device == device and t.is_contiguous()
+                   and (n is None or t.numel() >= n), f"{name} must be int32 [{n}] on the device")
+            return t.data_ptr()
+
+        wph = arr(self.window_per_head, num_q_heads, "window_per_head")
+        if self.kind == L.PKV_MASK_PREFIX_LM:
+            _check(self.prefix_len is not None, "prefix-LM mask needs prefix_len")
+        if self.kind == L.PKV_MASK_DOCUMENT:
+            _check(self.doc_offsets is not None and self.doc_starts is not None,
+                   "document mask needs doc_offsets and doc_starts")
+        return L.MaskModC(int(self.kind), int(self.window),
+                          arr(self.window_per_seq, batch, "window_per_seq"), wph,
+                          arr(self.prefix_len, batch, "prefix_len"),
+                          arr(self.doc_offsets, batch + 1, "doc_offsets"),
+                          arr(self.doc_starts, None, "doc_starts"))
 
 
 def no_mask() -> MaskMod:
@@ -53,10 +76,22 @@ def causal() -> MaskMod:
     return MaskMod(L.PKV_MASK_CAUSAL)
 
 
-def sliding_window(window: Union[int, torch.Tensor]) -> MaskMod:
+def sliding_window(window: Union[int, torch.Tensor], per_head: Optional[torch.Tensor] = None
+                   ) -> MaskMod:
+    """Sliding window: a scalar, a per-sequence tensor, and/or per-head windows."""
     if isinstance(window, torch.Tensor):
-        return MaskMod(L.PKV_MASK_SLIDING, 0, window)
-    return MaskMod(L.PKV_MASK_SLIDING, int(window))
+        return MaskMod(L.PKV_MASK_SLIDING, 0, window, per_head)
+    return MaskMod(L.PKV_MASK_SLIDING, int(window), None, per_head)
+
+
+def prefix_lm(prefix_len: torch.Tensor) -> MaskMod:
+    """Bidirectional prefix of ``prefix_len[b]`` keys, causal after it."""
+    return MaskMod(L.PKV_MASK_PREFIX_LM, prefix_len=prefix_len)
+
+
+def document(doc_offsets: torch.Tensor, doc_starts: torch.Tensor) -> MaskMod:
+    """Causal within documents packed into each sequence (CSR of start positions)."""
+    return MaskMod(L.PKV_MASK_DOCUMENT, doc_offsets=doc_offsets, doc_starts=doc_starts)
 
 
 def _check(cond, msg):
@@ -177,7 +212,7 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, seq_lens, scale=No
         workspace = decode_workspace(B, Hq, k_cache)
     L.check(L.lib().paged_attention_decode(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), cache_desc(k_cache), _ptr(block_tables),
-        block_tables.shape[1], _ptr(seq_lens), B, Hq, float(scale), mask_mod.to_c(B, dev),
+        block_tables.shape[1], _ptr(seq_lens), B, Hq, float(scale), mask_mod.to_c(B, dev, Hq),
         _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _ptr(dbg_err), _stream()))
     return out, lse
 
@@ -227,7 +262,7 @@ def paged_attention_decode_shared_prefix(q, k_cache, v_cache, block_tables, seq_
         workspace = shared_prefix_workspace(B, Hq, k_cache)
     L.check(L.lib().paged_attention_decode_shared_prefix(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), cache_desc(k_cache), _ptr(block_tables),
-        block_tables.shape[1], _ptr(seq_lens), B, Hq, float(scale), mask_mod.to_c(B, dev),
+        block_tables.shape[1], _ptr(seq_lens), B, Hq, float(scale), mask_mod.to_c(B, dev, Hq),
         _ptr(group_start), group_start.numel() - 1, int(max_group_size), _ptr(shared_len),
         _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _ptr(dbg_err), _stream()))
     return out, lse
@@ -260,7 +295,7 @@ def paged_attention_prefill(q, k_new, v_new, k_cache, v_cache, block_tables, ctx
     L.check(L.lib().paged_attention_prefill(
         _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), cache_desc(k_cache),
         _ptr(block_tables), block_tables.shape[1], _ptr(ctx_lens), _ptr(q_lens), B, T, Hq,
-        float(scale) if scale is not None else 0.0, mask_mod.to_c(B, dev), _ptr(out), _ptr(lse),
+        float(scale) if scale is not None else 0.0, mask_mod.to_c(B, dev, Hq), _ptr(out), _ptr(lse),
         _ptr(dbg_err), _stream()))
     return out, lse
 

@@ -17,17 +17,31 @@ LSE_ATOL = 1e-3
 NORM_RTOL = 1e-2
 
 
+MASK_EXTRA = ("window_per_head", "prefix_len", "doc_offsets", "doc_starts")
+
+
 def to_dev(case, dev):
     d = {}
     for name in ("k_cache", "v_cache", "block_tables", "seq_lens", "q", "k_new", "v_new",
                  "slot_mapping", "ctx_lens", "q_lens", "window_per_seq"):
         t = getattr(case, name)
         d[name] = None if t is None else t.to(dev).contiguous()
+    extra = case.extra.get("mask", {})
+    for name in MASK_EXTRA:
+        t = extra.get(name)
+        d[name] = None if t is None else t.to(dev).contiguous()
     return d
 
 
 def mask_of(case, dev_tensors):
-    return pkv.MaskMod(case.mask_kind, case.window, dev_tensors["window_per_seq"])
+    return pkv.MaskMod(case.mask_kind, case.window, dev_tensors["window_per_seq"],
+                       *(dev_tensors.get(n) for n in MASK_EXTRA))
+
+
+def mask_kwargs(case):
+    """The further mask arguments of the oracle calls (CPU tensors or None)."""
+    extra = case.extra.get("mask", {})
+    return {n: extra.get(n) for n in MASK_EXTRA}
 
 
 def assert_attention_close(out, lse, ref_out, ref_lse, dtype, what=""):
@@ -81,6 +95,8 @@ def oracle_after_append(case):
 def oracle_decode(case, kc, vc, rows=None):
     if rows is None:
         return oracle.paged_decode(case.q, kc, vc, case.block_tables, case.seq_lens, case.scale,
-                                   case.mask_kind, case.window, case.window_per_seq)
+                                   case.mask_kind, case.window, case.window_per_seq,
+                                   **mask_kwargs(case))
     return oracle.paged_decode_rows(case.q, kc, vc, case.block_tables, case.seq_lens, case.scale,
-                                    case.mask_kind, case.window, case.window_per_seq, rows=rows)
+                                    case.mask_kind, case.window, case.window_per_seq, rows=rows,
+                                    **mask_kwargs(case))

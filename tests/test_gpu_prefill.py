@@ -16,7 +16,7 @@ import torch
 import oracle
 import paged_kv_cache_gather_b200 as pkv
 from paged_kv_cache_gather_b200 import inputs as I
-from parity import assert_attention_close, mask_of, to_dev
+from parity import assert_attention_close, mask_kwargs, mask_of, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -41,8 +41,9 @@ def check_full(case, dev):
     ref_o, ref_l = oracle.paged_prefill(case.q, case.k_new, case.v_new, case.k_cache,
                                         case.v_cache, case.block_tables, case.ctx_lens,
                                         case.q_lens, case.scale, case.mask_kind, case.window,
-                                        case.window_per_seq)
+                                        case.window_per_seq, **mask_kwargs(case))
     assert_attention_close(out, lse, ref_o, ref_l, torch.bfloat16, case.name)
+    return out, lse
 
 
 SMALL = [
