@@ -68,6 +68,8 @@ extern "C" {
 #define PKV_DBG_LENGTH 4      /* a length needs more table entries than given */
 #define PKV_DBG_TIMEOUT 8     /* a bounded wait on a copy gave up */
 #define PKV_DBG_QLEN_SUM 16   /* prefill: sum of q_lens differs from total_q */
+#define PKV_DBG_OUT_OF_BLOCKS 32  /* reserve: too few free blocks, or a bad free stack */
+#define PKV_DBG_REFCOUNT 64   /* reserve: a block held by more sequences than its refcount */
 
 typedef enum { PKV_F32 = 0, PKV_BF16 = 1 } pkv_dtype;
 
@@ -165,6 +167,50 @@ PKV_API int paged_kv_gather(const void* k_cache, const void* v_cache, pkv_cache_
 PKV_API int paged_kv_copy_blocks(void* k_cache, void* v_cache, pkv_cache_desc cache,
                                  const int32_t* block_pairs, int32_t num_pairs,
                                  int32_t* dbg_err, void* stream);
+
+/*
+ * paged_kv_reserve_slots — device-side block allocation for an append step:
+ * slots for the new tokens, new blocks from a free stack, copy-on-write of
+ * shared partly filled blocks; no host round trip (CUDA-graph capturable).
+ * Source: "Ultimate Guide to PagedAttention": dynamic growth (a request whose
+ * last block is full takes a free block and appends it to its table) and
+ * memory sharing (blocks of a common prefix are held with a reference count
+ * and copied when one of their holders writes to them).
+ * The result is that of serving the sequences one by one in batch order:
+ * sequence b reserves positions seq_lens[b] .. seq_lens[b]+num_new[b]-1; if
+ * the first of them falls in its partly filled last block and that block is
+ * shared (refcount > 1), the sequence first takes a private copy of it (the
+ * old block's refcount drops by one; when every holder of the block appends
+ * in the same call, the last holder in batch order keeps the block); each
+ * further block it grows into is taken from the free stack. Blocks are taken
+ * from the top of the stack in that order.
+ *   block_tables   int32 [batch, max_blocks_per_seq], updated in place.
+ *   seq_lens       int32 [batch]: lengths before; on success += num_new.
+ *   num_new        int32 [batch] >= 0.
+ *   free_stack     int32 [num_blocks]: free block ids; the top is
+ *   free_top       free_stack[*free_top - 1]; *free_top (int32) is updated.
+ *   refcount       int32 [num_blocks]: holders of each block, updated (taken
+ *                  blocks get 1).
+ *   scratch        int32 [2 * num_blocks] (paged_kv_reserve_scratch_size()
+ *                  bytes), zero before the first call; every call leaves it zero.
+ *   slot_mapping   out int64 [num_tokens], num_tokens = sum of num_new: the
+ *                  new tokens' slots, sequence by sequence (the slot_mapping of
+ *                  paged_kv_append).
+ *   cow_pairs      out int32 [batch, 2]: (src, dst) of the copy sequence b made,
+ *                  (-1, -1) if none. The copies of K and V happen in this call.
+ * All arrays are device memory. If the free stack holds too few blocks, a
+ * table is too narrow, a block id is outside the pool, a refcount is below
+ * the number of holders, or num_tokens differs from the sum, nothing changes,
+ * every slot is -1 and a PKV_DBG_* bit is set in dbg_err. batch <= 8192.
+ * Three kernel launches on `stream`.
+ */
+PKV_API size_t paged_kv_reserve_scratch_size(pkv_cache_desc cache);
+PKV_API int paged_kv_reserve_slots(void* k_cache, void* v_cache, pkv_cache_desc cache,
+                                   int32_t* block_tables, int32_t max_blocks_per_seq,
+                                   int32_t* seq_lens, const int32_t* num_new, int32_t batch,
+                                   int32_t* free_stack, int32_t* free_top, int32_t* refcount,
+                                   int32_t* scratch, int64_t* slot_mapping, int32_t num_tokens,
+                                   int32_t* cow_pairs, int32_t* dbg_err, void* stream);
 
 /*
  * paged_attention_decode_workspace_size — bytes of scratch the decode call
@@ -280,6 +326,29 @@ PKV_API int paged_attention_decode_shared_prefix(
     const int32_t* group_start, int32_t num_groups, int32_t max_group_size,
     const int32_t* shared_len, void* out, float* lse, void* workspace, size_t workspace_bytes,
     int32_t* dbg_err, void* stream);
+
+/*
+ * paged_attention_block_mask — the block-sparse table of a mask modifier.
+ * Source: "Paged Attention Meets FlexAttention" (abstract): FlexAttention mask
+ * modifiers applied inside the paged kernel, which skips blocks no query of
+ * a tile can see. The attention calls derive these classes themselves; this
+ * call writes them out (for inspection, for planning work, for tests).
+ * Sequence b has ctx_lens[b] keys before q_lens[b] queries at positions
+ * ctx_lens[b] + i, and ctx_lens[b] + q_lens[b] keys in all (a decode step is
+ * ctx = seq_len - 1, q = 1). For query head h, query tile qt (queries
+ * qt*q_tile .. qt*q_tile+q_tile-1 of the sequence's q_lens[b]) and key tile kt
+ * (keys kt*k_tile .. kt*k_tile+k_tile-1), out[((b*num_q_heads + h)*n_q_tiles
+ * + qt)*n_k_tiles + kt] is PKV_BLOCK_SKIP (no pair visible, or the tile lies
+ * past the sequence), PKV_BLOCK_PARTIAL or PKV_BLOCK_FULL (every pair visible).
+ *   ctx_lens, q_lens  device int32 [batch]; out  device uint8, written in full.
+ */
+#define PKV_BLOCK_SKIP 0
+#define PKV_BLOCK_PARTIAL 1
+#define PKV_BLOCK_FULL 2
+PKV_API int paged_attention_block_mask(const int32_t* ctx_lens, const int32_t* q_lens,
+                                       int32_t batch, int32_t num_q_heads, pkv_mask_mod mask,
+                                       int32_t q_tile, int32_t k_tile, int32_t n_q_tiles,
+                                       int32_t n_k_tiles, uint8_t* out, void* stream);
 
 /*
  * paged_attention_decode_noalloc — paged_attention_decode without a

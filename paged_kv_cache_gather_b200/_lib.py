@@ -23,6 +23,8 @@ PKV_DBG_SLOT = 2
 PKV_DBG_LENGTH = 4
 PKV_DBG_TIMEOUT = 8
 PKV_DBG_QLEN_SUM = 16
+PKV_DBG_OUT_OF_BLOCKS = 32
+PKV_DBG_REFCOUNT = 64
 
 PKV_F32 = 0
 PKV_BF16 = 1
@@ -32,6 +34,10 @@ PKV_MASK_CAUSAL = 1
 PKV_MASK_SLIDING = 2
 PKV_MASK_PREFIX_LM = 3
 PKV_MASK_DOCUMENT = 4
+
+PKV_BLOCK_SKIP = 0
+PKV_BLOCK_PARTIAL = 1
+PKV_BLOCK_FULL = 2
 
 # every symbol the header declares; the CPU test checks that all are exported
 EXPORTS = (
@@ -44,6 +50,9 @@ EXPORTS = (
     "paged_attention_decode_noalloc",
     "paged_attention_decode_shared_prefix_workspace_size",
     "paged_attention_decode_shared_prefix",
+    "paged_attention_block_mask",
+    "paged_kv_reserve_scratch_size",
+    "paged_kv_reserve_slots",
     "pkv_debug_exp2",
     "pkv_status_string",
     "pkv_last_error",
@@ -105,6 +114,14 @@ def _declare(lib):
         _vp, _vp, _vp, CacheDescC, _vp, _i32, _vp, _i32, _i32, _f32, MaskModC, _vp, _i32, _i32,
         _vp, _vp, _vp, _vp, _sz, _vp, _vp]
     lib.paged_attention_decode_shared_prefix.restype = ctypes.c_int
+    lib.paged_attention_block_mask.argtypes = [_vp, _vp, _i32, _i32, MaskModC, _i32, _i32, _i32,
+                                               _i32, _vp, _vp]
+    lib.paged_attention_block_mask.restype = ctypes.c_int
+    lib.paged_kv_reserve_scratch_size.argtypes = [CacheDescC]
+    lib.paged_kv_reserve_scratch_size.restype = _sz
+    lib.paged_kv_reserve_slots.argtypes = [_vp, _vp, CacheDescC, _vp, _i32, _vp, _vp, _i32, _vp,
+                                           _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp]
+    lib.paged_kv_reserve_slots.restype = ctypes.c_int
     lib.pkv_debug_exp2.argtypes = [_vp, _vp, _i32, _vp]
     lib.pkv_debug_exp2.restype = ctypes.c_int
     lib.pkv_status_string.argtypes = [ctypes.c_int]

@@ -84,14 +84,16 @@ __global__ void __launch_bounds__(256) kv_gather_kernel(
 
 // Copy-on-write: block pairs (src, dst); every KV head's rows of block src
 // are copied to block dst, K and V. One thread per 16-byte vector.
+// With `skip_unset`, pairs (-1, -1) are holes in the list and copy nothing.
 __global__ void __launch_bounds__(256) kv_copy_blocks_kernel(
     int4* __restrict__ k_cache, int4* __restrict__ v_cache, const int32_t* __restrict__ pairs,
-    int64_t num_vec, int64_t vec_per_block, int32_t num_blocks, int32_t* dbg) {
+    int64_t num_vec, int64_t vec_per_block, int32_t num_blocks, bool skip_unset, int32_t* dbg) {
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < num_vec; i += stride) {
     const int64_t pr = i / vec_per_block;
     const int64_t off = i - pr * vec_per_block;
     const int32_t src = __ldg(pairs + 2 * pr), dst = __ldg(pairs + 2 * pr + 1);
+    if (skip_unset && src == -1 && dst == -1) continue;
     if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
       if (off == 0) flag_error(dbg, PKV_DBG_BLOCK_ID);
       continue;
@@ -141,7 +143,8 @@ int launch_gather(const void* k_cache, const void* v_cache, const pkv_cache_desc
 }
 
 int launch_copy_blocks(void* k_cache, void* v_cache, const pkv_cache_desc& c,
-                       const int32_t* pairs, int32_t num_pairs, int32_t* dbg, cudaStream_t s) {
+                       const int32_t* pairs, int32_t num_pairs, int32_t* dbg, cudaStream_t s,
+                       bool skip_unset) {
   const int es = dtype_size(c.dtype);
   const int64_t vec_per_block = (int64_t)c.num_kv_heads * c.block_size * c.head_dim * es / 16;
   const int64_t num_vec = (int64_t)num_pairs * vec_per_block;
@@ -149,7 +152,7 @@ int launch_copy_blocks(void* k_cache, void* v_cache, const pkv_cache_desc& c,
   const int threads = 256;
   kv_copy_blocks_kernel<<<grid_for(num_vec, threads), threads, 0, s>>>(
       static_cast<int4*>(k_cache), static_cast<int4*>(v_cache), pairs, num_vec, vec_per_block,
-      c.num_blocks, dbg);
+      c.num_blocks, skip_unset, dbg);
   return check_launch("paged_kv_copy_blocks");
 }
 

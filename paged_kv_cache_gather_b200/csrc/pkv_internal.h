@@ -41,8 +41,10 @@ int launch_gather(const void* k_cache, const void* v_cache, const pkv_cache_desc
                   const int32_t* tables, int32_t max_blocks, const int32_t* lens, int32_t batch,
                   int32_t out_max_len, void* k_out, void* v_out, int32_t* dbg, cudaStream_t s);
 
+// With skip_unset, pairs (-1, -1) copy nothing (a list with holes).
 int launch_copy_blocks(void* k_cache, void* v_cache, const pkv_cache_desc& c,
-                       const int32_t* pairs, int32_t num_pairs, int32_t* dbg, cudaStream_t s);
+                       const int32_t* pairs, int32_t num_pairs, int32_t* dbg, cudaStream_t s,
+                       bool skip_unset = false);
 
 struct DecodeArgs {
   const void* q;

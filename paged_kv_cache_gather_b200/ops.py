@@ -11,6 +11,7 @@ import math
 from dataclasses import dataclass
 from typing import Optional, Union
 
+import numpy as np
 import torch
 
 from . import _lib as L
@@ -298,6 +299,77 @@ def paged_attention_prefill(q, k_new, v_new, k_cache, v_cache, block_tables, ctx
         float(scale) if scale is not None else 0.0, mask_mod.to_c(B, dev, Hq), _ptr(out), _ptr(lse),
         _ptr(dbg_err), _stream()))
     return out, lse
+
+
+@dataclass
+class DevicePool:
+    """Device-side allocation state of one KV pool: a free stack (top at
+    ``free_stack[free_top - 1]``), per-block reference counts and the scratch
+    the reserve call keeps at zero. ``from_manager`` copies a host
+    ``BlockManager``'s state (its free list pops from the end, as here)."""
+
+    free_stack: torch.Tensor   # int32 [num_blocks]
+    free_top: torch.Tensor     # int32 [1]
+    refcount: torch.Tensor     # int32 [num_blocks]
+    scratch: torch.Tensor      # int32 [2 * num_blocks], zero
+
+    @staticmethod
+    def from_manager(mgr, device):
+        nb = mgr.num_blocks
+        stack = torch.zeros(nb, dtype=torch.int32)
+        free = list(mgr._free)
+        if free:
+            stack[:len(free)] = torch.tensor(free, dtype=torch.int32)
+        return DevicePool(stack.to(device), torch.tensor([len(free)], dtype=torch.int32,
+                                                         device=device),
+                          torch.from_numpy(mgr.refcount.astype(np.int32)).to(device),
+                          torch.zeros(2 * nb, dtype=torch.int32, device=device))
+
+
+def paged_kv_reserve_slots(k_cache, v_cache, block_tables, seq_lens, num_new, pool: DevicePool,
+                           num_tokens, dbg_err=None):
+    """Reserve slots for ``num_new[b]`` new tokens of every sequence on the
+    device (new blocks from the pool, copy-on-write of shared partly filled
+    blocks). Updates block_tables, seq_lens and the pool in place. Returns
+    (slot_mapping int64 [num_tokens], cow_pairs int32 [B, 2])."""
+    _check_pool(k_cache, v_cache)
+    dev = k_cache.device
+    for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens"), (num_new, "num_new"),
+                    (pool.free_stack, "free_stack"), (pool.free_top, "free_top"),
+                    (pool.refcount, "refcount"), (pool.scratch, "scratch")):
+        _i32(t, name, dev)
+    B = seq_lens.numel()
+    _check(block_tables.dim() == 2 and block_tables.shape[0] == B and num_new.numel() == B,
+           "block_tables [B, M], seq_lens [B] and num_new [B] must agree")
+    nb = k_cache.shape[0]
+    _check(pool.free_stack.numel() >= nb and pool.refcount.numel() >= nb and
+           pool.scratch.numel() >= 2 * nb, "pool arrays are smaller than the pool")
+    slots = torch.empty(max(int(num_tokens), 1), dtype=torch.int64, device=dev)
+    pairs = torch.empty(B, 2, dtype=torch.int32, device=dev)
+    L.check(L.lib().paged_kv_reserve_slots(
+        _ptr(k_cache), _ptr(v_cache), cache_desc(k_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(seq_lens), _ptr(num_new), B, _ptr(pool.free_stack),
+        _ptr(pool.free_top), _ptr(pool.refcount), _ptr(pool.scratch), _ptr(slots),
+        int(num_tokens), _ptr(pairs), _ptr(dbg_err), _stream()))
+    return slots[:int(num_tokens)], pairs
+
+
+def block_mask(ctx_lens, q_lens, num_q_heads, mask_mod: MaskMod, q_tile=128, k_tile=128):
+    """Block-sparse table of a mask: uint8 [B, Hq, n_q_tiles, n_k_tiles] with
+    0 = skipped, 1 = partial, 2 = every pair visible (see the C header)."""
+    dev = ctx_lens.device
+    _i32(ctx_lens, "ctx_lens", dev)
+    _i32(q_lens, "q_lens", dev)
+    B = ctx_lens.numel()
+    _check(q_lens.numel() == B, "ctx_lens and q_lens must agree on the batch")
+    n_q = int(q_lens.max().item()) if B else 0
+    n_k = int((ctx_lens + q_lens).max().item()) if B else 0
+    nqt, nkt = -(-n_q // q_tile), -(-n_k // k_tile)
+    out = torch.empty(B, num_q_heads, nqt, nkt, dtype=torch.uint8, device=dev)
+    L.check(L.lib().paged_attention_block_mask(
+        _ptr(ctx_lens), _ptr(q_lens), B, num_q_heads, mask_mod.to_c(B, dev, num_q_heads),
+        int(q_tile), int(k_tile), nqt, nkt, _ptr(out), _stream()))
+    return out
 
 
 def read_dbg(dbg_err):
