@@ -58,12 +58,12 @@ def peaks():
 # after any change to them the bench reports null until they are profiled again.
 PROFILED_TRAFFIC = {
     "decode": {"sources": ['csrc/decode.cu', 'csrc/pkv_common.cuh'],
-               "sha256": "4c37c4b9b05470cef1de74ba2b67369535fbe198e78a6f0b2b0c27b9c0491288",
-               "per_unit": 194804224 / 190134992,  # per algorithmic byte (16-seq ragged case)
+               "sha256": "4dfba94f197e0cc5773e7e7c5c22ea82355203cedb893f59034d2023ef227efb",
+               "per_unit": 194786816 / 190134992,  # per algorithmic byte (16-seq ragged case)
                },
     "prefill": {"sources": ['csrc/prefill.cu', 'csrc/pkv_common.cuh', 'csrc/tc_sm100.cuh'],
-                "sha256": "c512983f32c3b9e728518ba3b9d0fe44f058ca87beeaf776300f53053a4e4b78",
-                "per_unit": 298265088 / 1065168666624,  # per causal FLOP (1-seq case)
+                "sha256": "d616477bd29b665cc799fcd7a0501dd3188c257a24e0f406fc4e586759a4cab6",
+                "per_unit": 299987200 / 1065168666624,  # per causal FLOP (1-seq case)
                 },
 }
 
@@ -401,6 +401,35 @@ def shared_prefix(dev, flush):
     return out
 
 
+def shared_prefix_only(args, dev, rank):
+    """The grouped (shared-prefix) decode of the beams workload alone, cold L2
+    before every call: warm-up calls, then timed calls; prints one JSON line."""
+    import paged_kv_cache_gather_b200 as pkv
+    from paged_kv_cache_gather_b200 import inputs as I
+
+    c = I.config4(shared=True)
+    kc, vc = c.k_cache.to(dev), c.v_cache.to(dev)
+    q, tab, lens = c.q.to(dev), c.block_tables.to(dev), c.seq_lens.to(dev)
+    gs, sl = c.extra["group_start"].to(dev), c.extra["shared_len"].to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=dev)
+    ws = pkv.shared_prefix_workspace(q.shape[0], q.shape[1], kc)
+    call = lambda: pkv.paged_attention_decode_shared_prefix(
+        q, kc, vc, tab, lens, gs, sl, c.extra["max_group_size"], c.scale, pkv.causal(),
+        out=o, lse=lse, workspace=ws)
+    for _ in range(args.warmup):
+        call()
+    flush = l2_flush_buffer(dev)
+    ms = time_calls(call, args.steps, flush)
+    unique = c.extra["unique_blocks"] * 8 * 16 * 128 * 2 * 2
+    if rank == 0:
+        print(json.dumps({"workload": "shared-prefix beams (8 groups x 8 beams, 4096 shared + "
+                                      "256 own tokens, 32/8 heads, d128, bf16)",
+                          "us_per_call": round(ms * 1e3, 2), "unique_bytes": unique,
+                          "unique_GBps": round(unique / (ms * 1e-3) / 1e9, 1),
+                          "steps": args.steps, "warmup": args.warmup}))
+
+
 # ------------------------------------------------------------------ CPU baseline
 
 def oracle_decode_sample(budget_s=12.0, seed=None):
@@ -558,7 +587,10 @@ def main():
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="all", choices=["all", "decode", "prefill"])
+    ap.add_argument("--workload", default="all",
+                    choices=["all", "decode", "prefill", "shared_prefix"],
+                    help="shared_prefix: only the grouped decode of the beams workload "
+                         "(a side measurement, not the bench line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the batch-1 sweep and the shared-prefix measurement")
@@ -574,6 +606,10 @@ def main():
         return
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.workload == "shared_prefix":
+        shared_prefix_only(args, dev, rank)
+        barrier(ws)
+        return
     pk, pk_kind = peaks()
     total_steps = args.warmup + args.steps
     seed = 1237 + rank
