@@ -430,6 +430,120 @@ def shared_prefix_only(args, dev, rank):
                           "steps": args.steps, "warmup": args.warmup}))
 
 
+def mask_modifiers(dev, d=None):
+    """Throughput under the further mask modifiers: the long-context prefill with
+    packed documents (mean 4096 tokens) and with a prefix-LM prefix covering half
+    the chunk (FLOPs of visible pairs only), and the ragged decode batch with
+    per-head windows (4096 on even heads, none on odd; bytes of the keys read)."""
+    import paged_kv_cache_gather_b200 as pkv
+    from paged_kv_cache_gather_b200 import inputs as I
+
+    res = {}
+    pw = PrefillWork(dev, 1239)
+    c = pw.case
+    C = c.ctx_lens.numpy().astype(np.int64)
+    Q = c.q_lens.numpy().astype(np.int64)
+    off, st = I.document_starts((C + Q).tolist(), 77, mean_doc=4096)
+    pairs = 0
+    for b in range(len(C)):
+        starts = np.sort(st.numpy()[off[b]:off[b + 1]])
+        qpos = C[b] + np.arange(Q[b])
+        ds = starts[np.searchsorted(starts, qpos, side="right") - 1]
+        pairs += int((qpos - ds + 1).sum())
+    pw.mask = pkv.document(off.to(dev), st.to(dev))
+    pw.prefill()
+    ms = time_calls(pw.prefill, 5)
+    fl = 4.0 * c.head_dim * pairs * c.num_q_heads
+    res["prefill_documents"] = {"ms": round(ms, 3), "tflops": round(fl / (ms * 1e-3) / 1e12, 1),
+                                "visible_pairs_per_head": pairs,
+                                "documents": int(off[-1].item())}
+    plen = C + Q // 2
+    pairs = int(sum((np.maximum(C[b] + np.arange(Q[b]) + 1, plen[b])).sum() for b in range(len(C))))
+    pw.mask = pkv.prefix_lm(torch.from_numpy(plen.astype(np.int32)).to(dev))
+    pw.prefill()
+    ms = time_calls(pw.prefill, 5)
+    fl = 4.0 * c.head_dim * pairs * c.num_q_heads
+    res["prefill_prefix_lm"] = {"ms": round(ms, 3), "tflops": round(fl / (ms * 1e-3) / 1e12, 1)}
+    del pw
+    torch.cuda.empty_cache()
+    d = d if d is not None else I.config3()
+    kc, vc = d.k_cache.to(dev), d.v_cache.to(dev)
+    q, tab, lens = d.q.to(dev), d.block_tables.to(dev), d.seq_lens.to(dev)
+    wph = torch.tensor([4096 if h % 2 == 0 else 0 for h in range(d.num_q_heads)],
+                       dtype=torch.int32, device=dev)
+    ws = pkv.decode_workspace(q.shape[0], q.shape[1], kc)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=dev)
+    mm = pkv.sliding_window(0, per_head=wph)
+    call = lambda: pkv.paged_attention_decode(q, kc, vc, tab, lens, d.scale, mm, out=o, lse=lse,
+                                              workspace=ws)
+    call()
+    ms = time_calls(call, 20)
+    nbytes = int(d.seq_lens.numpy().astype(np.int64).sum()) * d.num_kv_heads * d.head_dim * 4
+    res["decode_per_head_windows"] = {"us": round(ms * 1e3, 1),
+                                      "GBps": round(nbytes / (ms * 1e-3) / 1e9, 1)}
+    return res
+
+
+def device_growth(dev, d=None):
+    """Device-side growth of the ragged decode batch (64 sequences, one token each):
+    the reserve call alone, and a whole step (reserve + append + decode) eager and
+    replayed from one CUDA graph."""
+    import paged_kv_cache_gather_b200 as pkv
+    from paged_kv_cache_gather_b200 import BlockManager
+    from paged_kv_cache_gather_b200 import inputs as I
+
+    d = d if d is not None else I.config3()
+    mgr = BlockManager(d.num_blocks, d.block_size, seed=3)
+    ids = list(range(d.batch))
+    for b, L in enumerate(d.seq_lens.tolist()):
+        mgr.add_sequence(b, L - 1)
+    width = d.block_tables.shape[1] + 8  # room for the ~70 steps taken here
+    tab = mgr.block_table_tensor(ids, width).to(dev)
+    lens = mgr.seq_lens_tensor(ids).to(dev)
+    pool = pkv.DevicePool.from_manager(mgr, dev)
+    kc, vc = d.k_cache.to(dev), d.v_cache.to(dev)
+    B = d.batch
+    one = torch.ones(B, dtype=torch.int32, device=dev)
+    kn, vn = d.k_new.to(dev), d.v_new.to(dev)
+    q = d.q.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, q.shape[1], dtype=torch.float32, device=dev)
+    ws = pkv.decode_workspace(B, q.shape[1], kc)
+
+    def reserve():
+        return pkv.paged_kv_reserve_slots(kc, vc, tab, lens, one, pool, B)[0]
+
+    def step():
+        slots = reserve()
+        pkv.paged_kv_append(kn, vn, slots, kc, vc)
+        pkv.paged_attention_decode(q, kc, vc, tab, lens, d.scale, pkv.causal(), out=o,
+                                   lse=lse, workspace=ws)
+
+    step()
+    us_res = time_calls(reserve, 20) * 1e3
+    us_eager = time_calls(step, 20) * 1e3
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            step()
+    torch.cuda.current_stream().wait_stream(s)
+    us_graph = time_calls(g.replay, 20) * 1e3
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g2, stream=s):
+            reserve()
+    torch.cuda.current_stream().wait_stream(s)
+    us_res_graph = time_calls(g2.replay, 20) * 1e3
+    del g, g2
+    return {"reserve_eager_us": round(us_res, 2), "reserve_graph_us": round(us_res_graph, 2),
+            "step_eager_us": round(us_eager, 1), "step_graph_us": round(us_graph, 1),
+            "batch": B, "free_blocks_left": int(pool.free_top.item()),
+            "note": "eager times include the Python binding's launch overhead"}
+
+
 # ------------------------------------------------------------------ CPU baseline
 
 def oracle_decode_sample(budget_s=12.0, seed=None):
@@ -761,6 +875,8 @@ def main():
         flush = l2_flush_buffer(dev)
         line["decode_sweep_batch1"] = decode_sweep(dev, flush)
         line["shared_prefix_beams"] = shared_prefix(dev, flush)
+        line["mask_modifiers"] = mask_modifiers(dev, dw.case)
+        line["device_growth"] = device_growth(dev, dw.case)
         del flush
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_decode_sample()

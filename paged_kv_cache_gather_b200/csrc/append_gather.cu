@@ -37,8 +37,10 @@ __global__ void __launch_bounds__(256) kv_append_kernel(
     const int64_t dst = (((blk * num_kv_heads + h) << block_shift) + row) * vec_per_row + c;
     const int4 kv = __ldg(k + i);
     const int4 vv = __ldg(v + i);
-    k_cache[dst] = kv;
-    v_cache[dst] = vv;
+    // streaming stores: the written rows leave L2 soon instead of lingering
+    // dirty until a later kernel's traffic evicts them
+    __stcs(k_cache + dst, kv);
+    __stcs(v_cache + dst, vv);
   }
 }
 

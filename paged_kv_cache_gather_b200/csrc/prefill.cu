@@ -660,7 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             v.y = pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
             v.z = pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
             v.w = pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-            *reinterpret_cast<uint4*>(dst + c * 32 + i) = v;
+            __stcs(reinterpret_cast<uint4*>(dst + c * 32 + i), v);  // streaming: leave L2 early
           }
         }
       }
