@@ -485,6 +485,43 @@ def mask_modifiers(dev, d=None):
     return res
 
 
+def fp8_decode(dev, d):
+    """The ragged decode batch on E4M3 pools: pools written by the quantising
+    append from the bf16 pools, then decode timed (20 calls, inputs > L2).
+    Reports the bytes read (codes + row scales) and the bf16-equivalent rate."""
+    import paged_kv_cache_gather_b200 as pkv
+
+    NB, Hkv, bs, D = d.k_cache.shape
+    kc = torch.empty(NB, Hkv, bs, D, dtype=torch.uint8, device=dev)
+    vc = torch.empty_like(kc)
+    ks = torch.empty(NB, Hkv, bs, dtype=torch.float32, device=dev)
+    vs = torch.empty_like(ks)
+    step = 4096  # blocks per append call
+    for b0 in range(0, NB, step):
+        b1 = min(NB, b0 + step)
+        rows_k = d.k_cache[b0:b1].to(dev).permute(0, 2, 1, 3).reshape(-1, Hkv, D).contiguous()
+        rows_v = d.v_cache[b0:b1].to(dev).permute(0, 2, 1, 3).reshape(-1, Hkv, D).contiguous()
+        slots = torch.arange(b0 * bs, b1 * bs, dtype=torch.int64, device=dev)
+        pkv.paged_kv_append_fp8(rows_k, rows_v, slots, kc, vc, ks, vs)
+    q, tab, lens = d.q.to(dev), d.block_tables.to(dev), d.seq_lens.to(dev)
+    wps = d.window_per_seq.to(dev)
+    mm = pkv.sliding_window(wps)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=dev)
+    ws = pkv.decode_workspace(q.shape[0], q.shape[1], kc)
+    call = lambda: pkv.paged_attention_decode_fp8(q, kc, vc, ks, vs, tab, lens, d.scale, mm,
+                                                  out=o, lse=lse, workspace=ws)
+    call()
+    ms = time_calls(call, 20)
+    vis = int(visible_tokens(d.seq_lens.numpy(), d.window_per_seq.numpy()).sum())
+    fp8_bytes = vis * Hkv * 2 * (D + 4)
+    bf16_bytes = vis * Hkv * 2 * D * 2
+    return {"us": round(ms * 1e3, 1), "bytes_read": fp8_bytes,
+            "GBps_read": round(fp8_bytes / (ms * 1e-3) / 1e9, 1),
+            "bf16_equivalent_GBps": round(bf16_bytes / (ms * 1e-3) / 1e9, 1),
+            "workload": "ragged decode batch (64 seqs, window 4096 on even), E4M3 pools"}
+
+
 def device_growth(dev, d=None):
     """Device-side growth of the ragged decode batch (64 sequences, one token each):
     the reserve call alone, and a whole step (reserve + append + decode) eager and
@@ -877,6 +914,7 @@ def main():
         line["shared_prefix_beams"] = shared_prefix(dev, flush)
         line["mask_modifiers"] = mask_modifiers(dev, dw.case)
         line["device_growth"] = device_growth(dev, dw.case)
+        line["fp8_decode"] = fp8_decode(dev, dw.case)
         del flush
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_decode_sample()

@@ -71,7 +71,10 @@ extern "C" {
 #define PKV_DBG_OUT_OF_BLOCKS 32  /* reserve: too few free blocks, or a bad free stack */
 #define PKV_DBG_REFCOUNT 64   /* reserve: a block held by more sequences than its refcount */
 
-typedef enum { PKV_F32 = 0, PKV_BF16 = 1 } pkv_dtype;
+/* PKV_FP8_E4M3: one-byte E4M3 codes (1 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits; largest finite value 448) with one float32 scale per stored
+ * row -- see paged_kv_append_fp8. */
+typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2 } pkv_dtype;
 
 typedef enum {
   PKV_MASK_NONE = 0,      /* every key of the sequence is visible */
@@ -139,6 +142,26 @@ typedef struct {
 PKV_API int paged_kv_append(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
                     void* k_cache, void* v_cache, pkv_cache_desc cache, int32_t* dbg_err,
                     void* stream);
+
+/*
+ * paged_kv_append_fp8 — write new tokens into E4M3 pools (quantised KV).
+ * The pages only gesture at compressing the KV cache, so the format is this
+ * library's reading: every stored row (one token's K or V for one KV head) has
+ * its own float32 scale s = amax / 448 (IEEE float32 division; 1 for an
+ * all-zero row), fixed when the row is written, and a value x is stored as the
+ * E4M3 code of x / s (IEEE division, round to nearest even, saturating at
+ * +-448); it reads back as code * s. Relative error <= 2^-4 for all but the
+ * smallest values of a row; no clipping, since every row sets its own scale.
+ *   k, v          [num_tokens, num_kv_heads, 128] BF16
+ *   k_cache, v_cache  E4M3 pools [num_blocks, num_kv_heads, block_size, 128] (1 byte each)
+ *   k_scale, v_scale  float32 [num_blocks, num_kv_heads, block_size]: row scales
+ *   slot_mapping  as for paged_kv_append.
+ * Supported: cache.dtype PKV_FP8_E4M3, head_dim 128.
+ */
+PKV_API int paged_kv_append_fp8(const void* k, const void* v, const int64_t* slot_mapping,
+                                int32_t num_tokens, void* k_cache, void* v_cache, float* k_scale,
+                                float* v_scale, pkv_cache_desc cache, int32_t* dbg_err,
+                                void* stream);
 
 /*
  * paged_kv_gather — resolve block tables into contiguous K and V.
@@ -248,6 +271,24 @@ PKV_API int paged_attention_decode(const void* q, const void* k_cache, const voi
                            int32_t num_q_heads, float scale, pkv_mask_mod mask, void* out,
                            float* lse, void* workspace, size_t workspace_bytes,
                            int32_t* dbg_err, void* stream);
+
+/*
+ * paged_attention_decode_fp8 — paged_attention_decode over E4M3 pools written
+ * by paged_kv_append_fp8 (half the bytes of bf16 per token). Same arguments,
+ * layouts, results and errors as paged_attention_decode, plus the row scales
+ * k_scale, v_scale (float32 [num_blocks, num_kv_heads, block_size], 16-byte
+ * aligned). q and out stay BF16; the result is attention over the decoded
+ * values code * scale. Codes are decoded exactly to f16 and the products run
+ * in f16 with float32 accumulation. Supported: head_dim 128, block_size >= 8,
+ * query groups of 1..8 heads, every mask kind; |q| < 65504.
+ */
+PKV_API int paged_attention_decode_fp8(const void* q, const void* k_cache, const void* v_cache,
+                                       const float* k_scale, const float* v_scale,
+                                       pkv_cache_desc cache, const int32_t* block_tables,
+                                       int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                       int32_t batch, int32_t num_q_heads, float scale,
+                                       pkv_mask_mod mask, void* out, float* lse, void* workspace,
+                                       size_t workspace_bytes, int32_t* dbg_err, void* stream);
 
 /*
  * paged_attention_prefill — a chunk of new query tokens per sequence over the

@@ -116,3 +116,13 @@ def kv_append_fp8(k, v, slot_mapping, k_codes, v_codes, k_scale, v_scale):
 def dequantize_pool(codes, scales):
     """float64 values of an E4M3 pool: decode(code) * scale of its row."""
     return decode_e4m3(codes) * np.asarray(scales, dtype=np.float64)[..., None]
+
+
+def quantize_rows(x):
+    """Vectorised ``quantize_row`` over the last axis: (codes uint8, scales float32)."""
+    xf = np.asarray(_f64(x), dtype=np.float32)
+    amax = np.max(np.abs(xf), axis=-1)
+    s = np.where(amax > 0, (amax / np.float32(E4M3_MAX)).astype(np.float32),
+                 np.float32(1.0)).astype(np.float32)
+    q = round_e4m3((xf / s[..., None]).astype(np.float32))
+    return encode_e4m3(q), s

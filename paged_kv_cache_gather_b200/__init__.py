@@ -4,6 +4,8 @@ Calls (thin bindings over the C ABI in ``include/pagedkv.h``):
 
 * ``paged_kv_append``         slot-mapped write of new tokens' K/V
 * ``paged_kv_gather``         block tables resolved to contiguous K/V
+* ``paged_kv_append_fp8`` / ``paged_attention_decode_fp8``  E4M3 pools with
+  per-row scales (half the bytes per token)
 * ``paged_kv_copy_blocks``    copy-on-write of shared blocks
 * ``paged_kv_reserve_slots``  device-side block allocation (growth + copy-on-write)
 * ``paged_attention_decode``  one query per sequence over paged KV
@@ -27,9 +29,11 @@ from .ops import (  # noqa: F401
     document,
     no_mask,
     paged_attention_decode,
+    paged_attention_decode_fp8,
     paged_attention_decode_shared_prefix,
     paged_attention_prefill,
     paged_kv_append,
+    paged_kv_append_fp8,
     paged_kv_copy_blocks,
     paged_kv_gather,
     paged_kv_reserve_slots,

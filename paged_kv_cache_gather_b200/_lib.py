@@ -28,6 +28,7 @@ PKV_DBG_REFCOUNT = 64
 
 PKV_F32 = 0
 PKV_BF16 = 1
+PKV_FP8_E4M3 = 2
 
 PKV_MASK_NONE = 0
 PKV_MASK_CAUSAL = 1
@@ -53,6 +54,8 @@ EXPORTS = (
     "paged_attention_block_mask",
     "paged_kv_reserve_scratch_size",
     "paged_kv_reserve_slots",
+    "paged_kv_append_fp8",
+    "paged_attention_decode_fp8",
     "pkv_debug_exp2",
     "pkv_status_string",
     "pkv_last_error",
@@ -122,6 +125,13 @@ def _declare(lib):
     lib.paged_kv_reserve_slots.argtypes = [_vp, _vp, CacheDescC, _vp, _i32, _vp, _vp, _i32, _vp,
                                            _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp]
     lib.paged_kv_reserve_slots.restype = ctypes.c_int
+    lib.paged_kv_append_fp8.argtypes = [_vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, CacheDescC, _vp,
+                                        _vp]
+    lib.paged_kv_append_fp8.restype = ctypes.c_int
+    lib.paged_attention_decode_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, CacheDescC, _vp, _i32,
+                                               _vp, _i32, _i32, _f32, MaskModC, _vp, _vp, _vp,
+                                               _sz, _vp, _vp]
+    lib.paged_attention_decode_fp8.restype = ctypes.c_int
     lib.pkv_debug_exp2.argtypes = [_vp, _vp, _i32, _vp]
     lib.pkv_debug_exp2.restype = ctypes.c_int
     lib.pkv_status_string.argtypes = [ctypes.c_int]

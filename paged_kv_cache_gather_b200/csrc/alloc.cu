@@ -257,6 +257,8 @@ PKV_API int paged_kv_reserve_slots(void* k_cache, void* v_cache, pkv_cache_desc 
   const char* fn = "paged_kv_reserve_slots";
   clear_last_error();
   if (int st = check_cache(cache, fn)) return st;
+  if (cache.dtype == PKV_FP8_E4M3)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: E4M3 pools (row scales) not supported", fn);
   if (batch < 0 || num_tokens < 0 || max_blocks_per_seq <= 0)
     return fail(PKV_ERR_INVALID_ARG, "%s: bad batch, num_tokens or max_blocks_per_seq", fn);
   if (batch > kMaxReserveBatch)

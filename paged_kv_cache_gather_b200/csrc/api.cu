@@ -73,6 +73,21 @@ bool make_pool_tensor_map(void* map_out, const void* base, int64_t rows, int32_t
   return r == CUDA_SUCCESS;
 }
 
+bool make_pool_tensor_map_u8(void* map_out, const void* base, int64_t rows, int32_t head_dim,
+                             int32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)head_dim};
+  cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(reinterpret_cast<CUtensorMap*>(map_out), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                  const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_tensor_map_bf16(void* map_out, const void* base, int rank, const uint64_t* dims,
                           const uint64_t* strides_bytes, const uint32_t* box) {
   auto fn = encode_fn();
@@ -98,7 +113,7 @@ int check_cache(const pkv_cache_desc& c, const char* fn) {
   if (c.block_size & (c.block_size - 1))
     return fail(PKV_ERR_INVALID_ARG, "%s: block_size %d is not a power of two", fn,
                 c.block_size);
-  if (c.dtype != PKV_F32 && c.dtype != PKV_BF16)
+  if (c.dtype != PKV_F32 && c.dtype != PKV_BF16 && c.dtype != PKV_FP8_E4M3)
     return fail(PKV_ERR_UNSUPPORTED, "%s: dtype %d not supported", fn, c.dtype);
   if ((c.head_dim * dtype_size(c.dtype)) % 16 != 0)
     return fail(PKV_ERR_UNSUPPORTED, "%s: head_dim*elem_size must be a multiple of 16 bytes",
@@ -146,6 +161,8 @@ int paged_kv_append(const void* k, const void* v, const int64_t* slot_mapping, i
                     void* stream) {
   g_last_error[0] = 0;
   if (int st = check_cache(cache, "paged_kv_append")) return st;
+  if (cache.dtype == PKV_FP8_E4M3)
+    return fail(PKV_ERR_UNSUPPORTED, "paged_kv_append: E4M3 pools take paged_kv_append_fp8");
   if (num_tokens < 0) return fail(PKV_ERR_INVALID_ARG, "paged_kv_append: num_tokens < 0");
   if (num_tokens == 0) return PKV_OK;
   if (!k || !v || !slot_mapping || !k_cache || !v_cache)
@@ -178,6 +195,8 @@ int paged_kv_copy_blocks(void* k_cache, void* v_cache, pkv_cache_desc cache,
                          void* stream) {
   g_last_error[0] = 0;
   if (int st = check_cache(cache, "paged_kv_copy_blocks")) return st;
+  if (cache.dtype == PKV_FP8_E4M3)
+    return fail(PKV_ERR_UNSUPPORTED, "paged_kv_copy_blocks: E4M3 pools (row scales) not supported");
   if (num_pairs < 0) return fail(PKV_ERR_INVALID_ARG, "paged_kv_copy_blocks: num_pairs < 0");
   if (num_pairs == 0) return PKV_OK;
   if (!k_cache || !v_cache || !block_pairs)
@@ -195,16 +214,20 @@ size_t paged_attention_decode_workspace_size(int32_t batch, int32_t num_q_heads,
   return decode_workspace_size(batch, num_q_heads, cache);
 }
 
-int paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
-                           pkv_cache_desc cache, const int32_t* block_tables,
-                           int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t batch,
-                           int32_t num_q_heads, float scale, pkv_mask_mod mask, void* out,
-                           float* lse, void* workspace, size_t workspace_bytes,
-                           int32_t* dbg_err, void* stream) {
+static int decode_entry(const char* fn, const void* q, const void* k_cache, const void* v_cache,
+                        const float* k_scale, const float* v_scale, pkv_cache_desc cache,
+                        const int32_t* block_tables, int32_t max_blocks_per_seq,
+                        const int32_t* seq_lens, int32_t batch, int32_t num_q_heads, float scale,
+                        pkv_mask_mod mask, void* out, float* lse, void* workspace,
+                        size_t workspace_bytes, int32_t* dbg_err, void* stream) {
   g_last_error[0] = 0;
-  const char* fn = "paged_attention_decode";
   if (int st = check_cache(cache, fn)) return st;
   if (int st = check_mask(mask, fn)) return st;
+  const bool fp8 = cache.dtype == PKV_FP8_E4M3;
+  if (fp8 != (k_scale != nullptr))
+    return fail(fp8 ? PKV_ERR_INVALID_ARG : PKV_ERR_UNSUPPORTED,
+                fp8 ? "%s: E4M3 pools need row scales" : "%s: %s", fn,
+                "row scales belong to E4M3 pools (paged_attention_decode_fp8)");
   if (batch < 0 || max_blocks_per_seq <= 0)
     return fail(PKV_ERR_INVALID_ARG, "%s: bad batch or max_blocks_per_seq", fn);
   if (num_q_heads <= 0 || num_q_heads % cache.num_kv_heads)
@@ -212,10 +235,11 @@ int paged_attention_decode(const void* q, const void* k_cache, const void* v_cac
                 num_q_heads, cache.num_kv_heads);
   if (!(scale == scale)) return fail(PKV_ERR_INVALID_ARG, "%s: scale is NaN", fn);
   if (batch == 0) return PKV_OK;
-  if (!q || !k_cache || !v_cache || !block_tables || !seq_lens || !out)
+  if (!q || !k_cache || !v_cache || !block_tables || !seq_lens || !out ||
+      (fp8 && (!k_scale || !v_scale)))
     return fail(PKV_ERR_INVALID_ARG, "%s: null pointer", fn);
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
-      !aligned16(workspace))
+      !aligned16(workspace) || (fp8 && (!aligned16(k_scale) || !aligned16(v_scale))))
     return fail(PKV_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", fn);
   const size_t need = decode_workspace_size(batch, num_q_heads, cache);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need))
@@ -224,7 +248,55 @@ int paged_attention_decode(const void* q, const void* k_cache, const void* v_cac
   DecodeArgs a{q,         k_cache, v_cache,    cache, block_tables, max_blocks_per_seq,
                seq_lens,  batch,   num_q_heads, scale, mask,         out,
                lse,       workspace, workspace_bytes, dbg_err, static_cast<cudaStream_t>(stream)};
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
   return launch_decode(a);
+}
+
+int paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
+                           pkv_cache_desc cache, const int32_t* block_tables,
+                           int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t batch,
+                           int32_t num_q_heads, float scale, pkv_mask_mod mask, void* out,
+                           float* lse, void* workspace, size_t workspace_bytes,
+                           int32_t* dbg_err, void* stream) {
+  return decode_entry("paged_attention_decode", q, k_cache, v_cache, nullptr, nullptr, cache,
+                      block_tables, max_blocks_per_seq, seq_lens, batch, num_q_heads, scale, mask,
+                      out, lse, workspace, workspace_bytes, dbg_err, stream);
+}
+
+int paged_attention_decode_fp8(const void* q, const void* k_cache, const void* v_cache,
+                               const float* k_scale, const float* v_scale, pkv_cache_desc cache,
+                               const int32_t* block_tables, int32_t max_blocks_per_seq,
+                               const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                               float scale, pkv_mask_mod mask, void* out, float* lse,
+                               void* workspace, size_t workspace_bytes, int32_t* dbg_err,
+                               void* stream) {
+  const char* fn = "paged_attention_decode_fp8";
+  if (cache.dtype != PKV_FP8_E4M3) {
+    g_last_error[0] = 0;
+    return fail(PKV_ERR_INVALID_ARG, "%s: the pool must be E4M3", fn);
+  }
+  return decode_entry(fn, q, k_cache, v_cache, k_scale, v_scale, cache, block_tables,
+                      max_blocks_per_seq, seq_lens, batch, num_q_heads, scale, mask, out, lse,
+                      workspace, workspace_bytes, dbg_err, stream);
+}
+
+int paged_kv_append_fp8(const void* k, const void* v, const int64_t* slot_mapping,
+                        int32_t num_tokens, void* k_cache, void* v_cache, float* k_scale,
+                        float* v_scale, pkv_cache_desc cache, int32_t* dbg_err, void* stream) {
+  g_last_error[0] = 0;
+  const char* fn = "paged_kv_append_fp8";
+  if (int st = check_cache(cache, fn)) return st;
+  if (cache.dtype != PKV_FP8_E4M3 || cache.head_dim != 128)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: E4M3 pools with head_dim 128 only", fn);
+  if (num_tokens < 0) return fail(PKV_ERR_INVALID_ARG, "%s: num_tokens < 0", fn);
+  if (num_tokens == 0) return PKV_OK;
+  if (!k || !v || !slot_mapping || !k_cache || !v_cache || !k_scale || !v_scale)
+    return fail(PKV_ERR_INVALID_ARG, "%s: null pointer", fn);
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PKV_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", fn);
+  return launch_append_fp8(k, v, slot_mapping, num_tokens, k_cache, v_cache, k_scale, v_scale,
+                           cache, dbg_err, static_cast<cudaStream_t>(stream));
 }
 
 int paged_attention_prefill(const void* q, const void* k_new, const void* v_new,

@@ -9,6 +9,8 @@
 // token goes to slot = block * block_size + row and nothing else moves.
 // Gather follows the block-table section of the same page: position p of
 // sequence b lives in block table[b][p / bs], row p % bs.
+#include <cuda_fp8.h>
+
 #include "pkv_common.cuh"
 #include "pkv_internal.h"
 
@@ -105,6 +107,64 @@ __global__ void __launch_bounds__(256) kv_copy_blocks_kernel(
   }
 }
 
+// E4M3 append: one warp per (token, KV head) row of K and of V; each lane
+// holds 4 of the 128 values. The row's scale is amax / 448 (IEEE float32
+// division; 1 for an all-zero row), each value is divided by it (IEEE) and
+// rounded to the nearest E4M3 code, ties to even, saturating at +-448.
+__device__ __forceinline__ uint32_t quantize4_e4m3(const uint2 w, float s) {
+  const float x0 = __uint_as_float(w.x << 16), x1 = __uint_as_float(w.x & 0xffff0000u);
+  const float x2 = __uint_as_float(w.y << 16), x3 = __uint_as_float(w.y & 0xffff0000u);
+  const __nv_fp8x2_storage_t lo =
+      __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(x0, s), __fdiv_rn(x1, s)), __NV_SATFINITE,
+                               __NV_E4M3);
+  const __nv_fp8x2_storage_t hi =
+      __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(x2, s), __fdiv_rn(x3, s)), __NV_SATFINITE,
+                               __NV_E4M3);
+  return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+__device__ __forceinline__ float row_amax(const uint2 w) {
+  float a = fmaxf(fmaxf(fabsf(__uint_as_float(w.x << 16)), fabsf(__uint_as_float(w.x & 0xffff0000u))),
+                  fmaxf(fabsf(__uint_as_float(w.y << 16)), fabsf(__uint_as_float(w.y & 0xffff0000u))));
+#pragma unroll
+  for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  return a;
+}
+
+__global__ void __launch_bounds__(256) kv_append_fp8_kernel(
+    const uint2* __restrict__ k, const uint2* __restrict__ v, const int64_t* __restrict__ slots,
+    int64_t rows, int32_t num_kv_heads, int32_t block_shift, int64_t pool_slots,
+    uint32_t* __restrict__ k_cache, uint32_t* __restrict__ v_cache, float* __restrict__ k_scale,
+    float* __restrict__ v_scale, int32_t* dbg) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int32_t bs_mask = (1 << block_shift) - 1;
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+       r += warps) {
+    const int64_t t = r / num_kv_heads;
+    const int64_t h = r - t * num_kv_heads;
+    const int64_t slot = __ldg(slots + t);
+    if (slot < 0) continue;
+    if (slot >= pool_slots) {
+      if (lane == 0) flag_error(dbg, PKV_DBG_SLOT);
+      continue;
+    }
+    const int64_t dst = (((slot >> block_shift) * num_kv_heads + h) << block_shift) + (slot & bs_mask);
+    // 128 bf16 values = 32 uint2 per row; 128 codes = 32 uint32 per row
+    const uint2 wk = __ldg(k + r * 32 + lane);
+    const uint2 wv = __ldg(v + r * 32 + lane);
+    const float ak = row_amax(wk), av = row_amax(wv);
+    const float sk = ak > 0.f ? __fdiv_rn(ak, 448.f) : 1.f;
+    const float sv = av > 0.f ? __fdiv_rn(av, 448.f) : 1.f;
+    __stcs(k_cache + dst * 32 + lane, quantize4_e4m3(wk, sk));
+    __stcs(v_cache + dst * 32 + lane, quantize4_e4m3(wv, sv));
+    if (lane == 0) {
+      k_scale[dst] = sk;
+      v_scale[dst] = sv;
+    }
+  }
+}
+
 static int grid_for(int64_t work, int threads) {
   const int sms = device_sm_count();
   int64_t blocks = (work + threads - 1) / threads;
@@ -127,6 +187,19 @@ int launch_append(const void* k, const void* v, const int64_t* slots, int32_t nu
       c.num_kv_heads, log2_int(c.block_size), (int64_t)c.num_blocks * c.block_size,
       static_cast<int4*>(k_cache), static_cast<int4*>(v_cache), dbg);
   return check_launch("paged_kv_append");
+}
+
+int launch_append_fp8(const void* k, const void* v, const int64_t* slots, int32_t num_tokens,
+                      void* k_cache, void* v_cache, float* k_scale, float* v_scale,
+                      const pkv_cache_desc& c, int32_t* dbg, cudaStream_t s) {
+  const int64_t rows = (int64_t)num_tokens * c.num_kv_heads;
+  if (rows == 0) return PKV_OK;
+  const int threads = 256;
+  kv_append_fp8_kernel<<<grid_for(rows * 32, threads), threads, 0, s>>>(
+      static_cast<const uint2*>(k), static_cast<const uint2*>(v), slots, rows, c.num_kv_heads,
+      log2_int(c.block_size), (int64_t)c.num_blocks * c.block_size,
+      static_cast<uint32_t*>(k_cache), static_cast<uint32_t*>(v_cache), k_scale, v_scale, dbg);
+  return check_launch("paged_kv_append_fp8");
 }
 
 int launch_gather(const void* k_cache, const void* v_cache, const pkv_cache_desc& c,

@@ -39,7 +39,7 @@ namespace pkv {
 constexpr int kTile = 16;            // tokens per tile
 constexpr int kMinTilesPerWorker = 2;
 constexpr int kWarpsPerCta = 12;     // default workers (warps) per CTA, one CTA per SM
-constexpr int kMaxWarpsPerCta = 12;  // largest built variant (sizes the workspace)
+constexpr int kMaxWarpsPerCta = 12;  // largest built bf16 variant (sizes the workspace)
 
 struct DecodeParams {
   const __nv_bfloat16* q;
@@ -54,6 +54,8 @@ struct DecodeParams {
   int32_t num_blocks;
   float scale_log2;    // scale * log2(e)
   pkv_mask_mod mask;
+  const float* k_scale;  // E4M3 pools: float32 scale of each stored row [pool rows]
+  const float* v_scale;
   __nv_bfloat16* out;
   float* lse;
   float* ws_o;         // [2 * workers, group, D] partial outputs (normalised)
@@ -173,20 +175,34 @@ __device__ __forceinline__ void cursor_advance(const DecodeParams& p, Cursor& c)
   }
 }
 
-template <int D>
+// Shared-memory layout. bf16 pools: a stage is a K tile then a V tile (16
+// rows x D, 128-byte-swizzled halves of 64 columns). E4M3 pools (KV8, D = 128):
+// a stage is a K tile then a V tile of 16 rows x 128 one-byte codes (one
+// swizzled 128-byte row per token), plus 128 bytes of row scales (K then V)
+// per stage, and each warp owns a f16 work tile that its V tile is decoded
+// into (same layout as a bf16 tile).
+template <int D, bool KV8 = false>
 struct Cfg {
-  static constexpr int kHalves = D / 64;                  // 128-byte column boxes per row
-  static constexpr int kTileBytes = kTile * D * 2;        // K (or V) bytes of one tile
-  static constexpr int kStageBytes = 2 * kTileBytes;      // K then V
+  static constexpr int kHalves = KV8 ? 1 : D / 64;            // TMA boxes per row
+  static constexpr int kTileBytes = kTile * D * (KV8 ? 1 : 2);  // K (or V) bytes of one tile
+  static constexpr int kStageBytes = 2 * kTileBytes;           // K then V
+  static constexpr int kWorkBytes = KV8 ? kTile * D * 2 : 0;
+  static constexpr int kScaleBytes = KV8 ? 2 * kTile * 4 : 0;
 };
 
 // PH: per-head sliding windows (each head column masks keys below its own
 // start); the instance without them carries none of that code.
-template <int D, int NSTAGE, int WPC, bool PH>
+// KV8: E4M3 pools with a float32 scale per stored row (D = 128). Codes are
+// decoded to f16 exactly (cvt.rn.f16x2.e4m3x2) and the MMAs run in f16: K's
+// row scales multiply the scores, V's row scales (times 256, which keeps the
+// products clear of f16 subnormals and is divided out at the end) multiply P.
+template <int D, int NSTAGE, int WPC, bool PH, bool KV8>
 __global__ void __launch_bounds__(WPC * 32, 1)
     decode_bf16_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, KV8>;
+  static_assert(!KV8 || D == 128, "E4M3 pools are built for head_dim 128");
+  constexpr float kVScale = 256.f;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzle atoms
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -194,7 +210,12 @@ __global__ void __launch_bounds__(WPC * 32, 1)
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   uint8_t* ring = smem + warp * NSTAGE * C::kStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + WPC * NSTAGE * C::kStageBytes) + warp * NSTAGE;
+  uint8_t* work = smem + WPC * NSTAGE * C::kStageBytes + warp * C::kWorkBytes;
+  float* scl = reinterpret_cast<float*>(smem + WPC * (NSTAGE * C::kStageBytes + C::kWorkBytes)) +
+               warp * NSTAGE * (C::kScaleBytes / 4);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+                       smem + WPC * (NSTAGE * (C::kStageBytes + C::kScaleBytes) + C::kWorkBytes)) +
+                   warp * NSTAGE;
 
   const int gw = blockIdx.x * WPC + warp;
   const bool writer = (gw == 0);
@@ -260,7 +281,7 @@ __global__ void __launch_bounds__(WPC * 32, 1)
           flag_error(p.dbg, PKV_DBG_BLOCK_ID);
           ids[pi] = 0;
         }
-        bytes += 2u * box_rows * D * 2;
+        bytes += KV8 ? 2u * box_rows * (D + 4) : 2u * box_rows * D * 2;
       }
     }
     fence_proxy_async_smem();
@@ -272,8 +293,13 @@ __global__ void __launch_bounds__(WPC * 32, 1)
 #pragma unroll
       for (int h = 0; h < C::kHalves; ++h) {
         const uint32_t o = h * (kTile * 128) + pi * box_rows * 128;
-        tma_load_2d_hint(kdst + o, &kmap, h * 64, row, bar, evict_first);
-        tma_load_2d_hint(vdst + o, &vmap, h * 64, row, bar, evict_first);
+        tma_load_2d_hint(kdst + o, &kmap, h * (KV8 ? 128 : 64), row, bar, evict_first);
+        tma_load_2d_hint(vdst + o, &vmap, h * (KV8 ? 128 : 64), row, bar, evict_first);
+      }
+      if constexpr (KV8) {
+        const uint32_t sdst = smem_u32(scl + stage * 2 * kTile) + pi * box_rows * 4;
+        bulk_load_1d(sdst, p.k_scale + row, box_rows * 4, bar);
+        bulk_load_1d(sdst + kTile * 4, p.v_scale + row, box_rows * 4, bar);
       }
     }
   };
@@ -324,8 +350,16 @@ __global__ void __launch_bounds__(WPC * 32, 1)
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         if (g4 < p.group) {
-          qf[kk][0] = __ldg(reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * c4));
-          qf[kk][1] = __ldg(reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + 2 * c4));
+          if constexpr (KV8) {
+            // f16 B fragments in the k order of the E4M3 A fragments: step kk
+            // covers columns 16kk..16kk+15, this lane's four at 16kk + 4*c4
+            const uint2 w = __ldg(reinterpret_cast<const uint2*>(qrow + kk * 16 + 4 * c4));
+            qf[kk][0] = pack_f16x2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u));
+            qf[kk][1] = pack_f16x2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+          } else {
+            qf[kk][0] = __ldg(reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * c4));
+            qf[kk][1] = __ldg(reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + 2 * c4));
+          }
         } else {
           qf[kk][0] = qf[kk][1] = 0u;
         }
@@ -346,14 +380,42 @@ __global__ void __launch_bounds__(WPC * 32, 1)
     const uint32_t parity = (uint32_t)((k / NSTAGE) & 1);
     uint8_t* kst = ring + stage * C::kStageBytes;
     const uint32_t kbase = smem_u32(kst);
-    const uint32_t vbase = kbase + C::kTileBytes;
+    const uint32_t vbase = KV8 ? smem_u32(work) : kbase + C::kTileBytes;
     if (!mbar_wait(smem_u32(bars + stage), parity)) {
       flag_error(p.dbg, PKV_DBG_TIMEOUT);
       return;
     }
     const int tok0 = (cur.s.t0 + (int)(cur.t - cur.seg_first)) * kTile;
     const bool partial = tok0 < cur.s.lo || tok0 + kTile > cur.s.hi;
-    if (partial) {
+    if constexpr (KV8) {
+      // decode the V codes into the f16 work tile (row r, 16-code chunks
+      // (lane & 1) * 4 ..); rows outside [lo, hi) become zero
+      const int r = lane >> 1;
+      const int pos = tok0 + r;
+      const bool live = pos >= cur.s.lo && pos < cur.s.hi;
+      const uint8_t* vrow = kst + C::kTileBytes + r * 128;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c8 = (lane & 1) * 4 + j;
+        const uint4 w = live ? *reinterpret_cast<const uint4*>(vrow + ((c8 ^ (r & 7)) << 4))
+                             : make_uint4(0u, 0u, 0u, 0u);
+        uint4 lo, hi;
+        lo.x = e4m3x2_to_f16x2(w.x);
+        lo.y = e4m3x2_to_f16x2(w.x >> 16);
+        lo.z = e4m3x2_to_f16x2(w.y);
+        lo.w = e4m3x2_to_f16x2(w.y >> 16);
+        hi.x = e4m3x2_to_f16x2(w.z);
+        hi.y = e4m3x2_to_f16x2(w.z >> 16);
+        hi.z = e4m3x2_to_f16x2(w.w);
+        hi.w = e4m3x2_to_f16x2(w.w >> 16);
+        const int c0 = 2 * c8, c1 = c0 + 1;  // f16 chunks of 8 values
+        *reinterpret_cast<uint4*>(work + (c0 >> 3) * (kTile * 128) + r * 128 +
+                                  (((c0 & 7) ^ (r & 7)) << 4)) = lo;
+        *reinterpret_cast<uint4*>(work + (c1 >> 3) * (kTile * 128) + r * 128 +
+                                  (((c1 & 7) ^ (r & 7)) << 4)) = hi;
+      }
+      __syncwarp();
+    } else if (partial) {
       // rows outside [lo, hi) may hold stale or non-finite data: zero them in V
       for (int i = lane; i < kTile * C::kHalves * 8; i += 32) {
         const int h = i / (kTile * 8);
@@ -371,22 +433,54 @@ __global__ void __launch_bounds__(WPC * 32, 1)
 
     // S^T (16 tokens x 8 heads) = K (16 x D) * Q^T (D x 8)
     float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (KV8) {
+      // one ldmatrix covers 32 codes of 16 rows; each 16-bit unit holds two
+      // codes, decoded into the f16 A fragments of two k16 steps whose k
+      // order the query fragments follow
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const int chunk = 2 * kk + kco;
-      const uint32_t addr = kbase + (chunk >> 3) * (kTile * 128) + krow * 128 +
-                            (((chunk & 7) ^ (krow & 7)) << 4);
-      uint32_t a[4];
-      ldmatrix_x4(a, addr);
-      if (kk & 1)
-        mma_bf16_16816(sb, a, qf[kk][0], qf[kk][1]);
-      else
-        mma_bf16_16816(sa, a, qf[kk][0], qf[kk][1]);
+      for (int s2 = 0; s2 < D / 32; ++s2) {
+        const int chunk = 2 * s2 + kco;
+        uint32_t r[4];
+        ldmatrix_x4(r, kbase + krow * 128 + ((chunk ^ (krow & 7)) << 4));
+        uint32_t a[4];
+        a[0] = e4m3x2_to_f16x2(r[0]);
+        a[1] = e4m3x2_to_f16x2(r[1]);
+        a[2] = e4m3x2_to_f16x2(r[0] >> 16);
+        a[3] = e4m3x2_to_f16x2(r[1] >> 16);
+        mma_f16_16816(sa, a, qf[2 * s2][0], qf[2 * s2][1]);
+        a[0] = e4m3x2_to_f16x2(r[2]);
+        a[1] = e4m3x2_to_f16x2(r[3]);
+        a[2] = e4m3x2_to_f16x2(r[2] >> 16);
+        a[3] = e4m3x2_to_f16x2(r[3] >> 16);
+        mma_f16_16816(sb, a, qf[2 * s2 + 1][0], qf[2 * s2 + 1][1]);
+      }
+    } else {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int chunk = 2 * kk + kco;
+        const uint32_t addr = kbase + (chunk >> 3) * (kTile * 128) + krow * 128 +
+                              (((chunk & 7) ^ (krow & 7)) << 4);
+        uint32_t a[4];
+        ldmatrix_x4(a, addr);
+        if (kk & 1)
+          mma_bf16_16816(sb, a, qf[kk][0], qf[kk][1]);
+        else
+          mma_bf16_16816(sa, a, qf[kk][0], qf[kk][1]);
+      }
     }
     // element e: token g4 (+8 for e >= 2), head 2*c4 + (e & 1)
     float x[4];
+    if constexpr (KV8) {
+      const float* ks = scl + stage * 2 * kTile;  // this tile's K row scales
+      const float k0 = ks[g4] * p.scale_log2, k1 = ks[g4 + 8] * p.scale_log2;
+      x[0] = (sa[0] + sb[0]) * k0;
+      x[1] = (sa[1] + sb[1]) * k0;
+      x[2] = (sa[2] + sb[2]) * k1;
+      x[3] = (sa[3] + sb[3]) * k1;
+    } else {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) x[e] = (sa[e] + sb[e]) * p.scale_log2;
+      for (int e = 0; e < 4; ++e) x[e] = (sa[e] + sb[e]) * p.scale_log2;
+    }
     if (partial) {
       const int p0 = tok0 + g4, p1 = p0 + 8;
       if (p0 < cur.s.lo || p0 >= cur.s.hi) x[0] = x[1] = -INFINITY;
@@ -431,8 +525,20 @@ __global__ void __launch_bounds__(WPC * 32, 1)
       }
     }
     // P^T rows (tokens) -> B operand (k = token, n = head) via 8x8 transposes
-    const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p00, p01));
-    const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p10, p11));
+    uint32_t pb0, pb1;
+    if constexpr (KV8) {
+      // V's row scale (x 256) joins P; rows outside [lo, hi) get 0, whatever
+      // their stored scale holds
+      const float* vs = scl + stage * 2 * kTile + kTile;
+      const int q0 = tok0 + g4, q1 = q0 + 8;
+      const float v0 = (q0 >= cur.s.lo && q0 < cur.s.hi) ? vs[g4] * kVScale : 0.f;
+      const float v1 = (q1 >= cur.s.lo && q1 < cur.s.hi) ? vs[g4 + 8] * kVScale : 0.f;
+      pb0 = movmatrix_trans(pack_f16x2(p00 * v0, p01 * v0));
+      pb1 = movmatrix_trans(pack_f16x2(p10 * v1, p11 * v1));
+    } else {
+      pb0 = movmatrix_trans(pack_bf16x2(p00, p01));
+      pb1 = movmatrix_trans(pack_bf16x2(p10, p11));
+    }
     // O^T (D x 8) += V^T (D x 16 tokens) * P^T (16 x 8)
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) {
@@ -441,7 +547,10 @@ __global__ void __launch_bounds__(WPC * 32, 1)
                             (((chunk & 7) ^ (vtok & 7)) << 4);
       uint32_t a[4];
       ldmatrix_x4_trans(a, addr);
-      mma_bf16_16816(o[mt], a, pb0, pb1);
+      if constexpr (KV8)
+        mma_f16_16816(o[mt], a, pb0, pb1);
+      else
+        mma_bf16_16816(o[mt], a, pb0, pb1);
     }
     __syncwarp();
 
@@ -456,7 +565,8 @@ __global__ void __launch_bounds__(WPC * 32, 1)
         s1 += __shfl_xor_sync(0xffffffffu, s1, off);
       }
       // a head that saw no key in this piece (per-head windows) gives 0, -inf
-      const float inv0 = s0 > 0.f ? 1.f / s0 : 0.f, inv1 = s1 > 0.f ? 1.f / s1 : 0.f;
+      const float un = KV8 ? 1.f / kVScale : 1.f;  // E4M3: O carries V's extra factor
+      const float inv0 = s0 > 0.f ? un / s0 : 0.f, inv1 = s1 > 0.f ? un / s1 : 0.f;
       const float lse0 = s0 > 0.f ? m0 * kLn2 + logf(s0) : -INFINITY;
       const float lse1 = s1 > 0.f ? m1 * kLn2 + logf(s1) : -INFINITY;
       const int h0 = 2 * c4, h1 = h0 + 1;
@@ -709,18 +819,20 @@ __global__ void __launch_bounds__(128) decode_f32_kernel(
 
 namespace {
 
-template <int D, int NSTAGE, int WPC, bool PH>
+template <int D, int NSTAGE, int WPC, bool PH, bool KV8 = false>
 int launch_bf16_impl(const DecodeArgs& a) {
-  using Cf = Cfg<D>;
+  using Cf = Cfg<D, KV8>;
   const int sms = device_sm_count();
   const int workers = sms * WPC;
   const int g = a.num_q_heads / a.cache.num_kv_heads;
-  const size_t smem = (size_t)WPC * NSTAGE * Cf::kStageBytes + WPC * NSTAGE * 8 + 1024;
+  const size_t smem =
+      (size_t)WPC * (NSTAGE * (Cf::kStageBytes + Cf::kScaleBytes) + Cf::kWorkBytes) +
+      WPC * NSTAGE * 8 + 1024;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(decode_bf16_kernel<D, NSTAGE, WPC, PH>,
+    if (cudaFuncSetAttribute(decode_bf16_kernel<D, NSTAGE, WPC, PH, KV8>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return check_launch("paged_attention_decode: smem attribute");
     attr_set[dev] = true;
@@ -728,9 +840,12 @@ int launch_bf16_impl(const DecodeArgs& a) {
   const int box_rows = a.cache.block_size >= kTile ? kTile : a.cache.block_size;
   const int64_t rows = (int64_t)a.cache.num_blocks * a.cache.num_kv_heads * a.cache.block_size;
   alignas(64) CUtensorMap kmap, vmap;
-  if (!make_pool_tensor_map(&kmap, a.k_cache, rows, D, box_rows) ||
-      !make_pool_tensor_map(&vmap, a.v_cache, rows, D, box_rows))
-    return fail(PKV_ERR_CUDA, "paged_attention_decode: tensor map encoding failed");
+  const bool maps_ok =
+      KV8 ? (make_pool_tensor_map_u8(&kmap, a.k_cache, rows, D, box_rows) &&
+             make_pool_tensor_map_u8(&vmap, a.v_cache, rows, D, box_rows))
+          : (make_pool_tensor_map(&kmap, a.k_cache, rows, D, box_rows) &&
+             make_pool_tensor_map(&vmap, a.v_cache, rows, D, box_rows));
+  if (!maps_ok) return fail(PKV_ERR_CUDA, "paged_attention_decode: tensor map encoding failed");
 
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
   DecodeParams p;
@@ -746,6 +861,8 @@ int launch_bf16_impl(const DecodeArgs& a) {
   p.num_blocks = a.cache.num_blocks;
   p.scale_log2 = a.scale * kLog2e;
   p.mask = a.mask;
+  p.k_scale = a.k_scale;
+  p.v_scale = a.v_scale;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.lse = a.lse;
   const size_t o_bytes = (size_t)2 * workers * g * D * 4;
@@ -756,7 +873,7 @@ int launch_bf16_impl(const DecodeArgs& a) {
   p.workers = workers;
   p.dbg = a.dbg;
 
-  decode_bf16_kernel<D, NSTAGE, WPC, PH><<<sms, WPC * 32, smem, a.stream>>>(kmap, vmap, p);
+  decode_bf16_kernel<D, NSTAGE, WPC, PH, KV8><<<sms, WPC * 32, smem, a.stream>>>(kmap, vmap, p);
   if (int st = check_launch("paged_attention_decode")) return st;
   const int64_t items = (int64_t)a.batch * a.cache.num_kv_heads * g;
   cudaLaunchConfig_t cfg = {};
@@ -786,9 +903,30 @@ int decode_warps_per_cta() {
   return w;
 }
 
+// Warps per CTA of the E4M3 decode (PKV_DECODE_FP8_WARPS picks another built
+// variant, for tuning sweeps).
+int decode_fp8_warps() {
+  static int w = [] {
+    const char* e = getenv("PKV_DECODE_FP8_WARPS");
+    int v = e ? atoi(e) : 16;
+    return v == 12 ? 12 : 16;  // 16 warps measured 9% faster on the ragged batch
+  }();
+  return w;
+}
+
 template <int D>
 int launch_bf16(const DecodeArgs& a) {
   // 192 KB of ring per CTA for head_dim 128 (8 KB stages), 160-192 KB for 64
+  if constexpr (D == 128) {
+    // E4M3 pools: 16 warps with 2-stage rings of 4 KB tiles (or 12 with 3) and
+    // a 4 KB work tile each, 197-201 KB per CTA
+    if (a.cache.dtype == PKV_FP8_E4M3) {
+      if (a.mask.kind == PKV_MASK_SLIDING && a.mask.window_per_head)
+        return launch_bf16_impl<D, 3, 12, true, true>(a);
+      if (decode_fp8_warps() == 16) return launch_bf16_impl<D, 2, 16, false, true>(a);
+      return launch_bf16_impl<D, 3, 12, false, true>(a);
+    }
+  }
   if (a.mask.kind == PKV_MASK_SLIDING && a.mask.window_per_head)
     return launch_bf16_impl<D, (D == 128 ? 2 : 4), 12, true>(a);
   switch (decode_warps_per_cta()) {
@@ -802,8 +940,9 @@ int launch_bf16(const DecodeArgs& a) {
 }  // namespace
 
 size_t decode_workspace_size(int32_t batch, int32_t num_q_heads, const pkv_cache_desc& c) {
-  if (c.dtype != PKV_BF16) return 0;
-  const int workers = device_sm_count() * kMaxWarpsPerCta;
+  if (c.dtype == PKV_F32) return 0;
+  // the E4M3 decode has a 16-warp variant
+  const int workers = device_sm_count() * (c.dtype == PKV_FP8_E4M3 ? 16 : kMaxWarpsPerCta);
   const int g = num_q_heads / c.num_kv_heads;
   const size_t o_bytes = (size_t)2 * workers * g * c.head_dim * 4;
   const size_t l_bytes = ((size_t)2 * workers * g * 4 + 255) & ~size_t(255);
@@ -825,6 +964,9 @@ int launch_decode(const DecodeArgs& a) {
         a.lse, a.dbg);
     return check_launch("paged_attention_decode (fp32)");
   }
+  if (a.cache.dtype == PKV_FP8_E4M3 && (a.cache.head_dim != 128 || !a.k_scale || !a.v_scale))
+    return fail(PKV_ERR_UNSUPPORTED,
+                "paged_attention_decode: E4M3 pools need head_dim 128 and row scales");
   if (g < 1 || g > 8)
     return fail(PKV_ERR_UNSUPPORTED, "paged_attention_decode: bf16 group size %d not in 1..8", g);
   if (a.cache.block_size < 8)

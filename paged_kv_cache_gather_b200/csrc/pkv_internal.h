@@ -25,7 +25,7 @@ int check_cache(const pkv_cache_desc& c, const char* fn);
 int check_mask(const pkv_mask_mod& m, const char* fn);
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-inline int dtype_size(int32_t dt) { return dt == PKV_BF16 ? 2 : 4; }
+inline int dtype_size(int32_t dt) { return dt == PKV_BF16 ? 2 : dt == PKV_FP8_E4M3 ? 1 : 4; }
 
 inline int log2_int(int32_t x) {
   int r = 0;
@@ -36,6 +36,11 @@ inline int log2_int(int32_t x) {
 int launch_append(const void* k, const void* v, const int64_t* slots, int32_t num_tokens,
                   void* k_cache, void* v_cache, const pkv_cache_desc& c, int32_t* dbg,
                   cudaStream_t s);
+
+// bf16 tokens quantised into E4M3 pools with a float32 scale per stored row.
+int launch_append_fp8(const void* k, const void* v, const int64_t* slots, int32_t num_tokens,
+                      void* k_cache, void* v_cache, float* k_scale, float* v_scale,
+                      const pkv_cache_desc& c, int32_t* dbg, cudaStream_t s);
 
 int launch_gather(const void* k_cache, const void* v_cache, const pkv_cache_desc& c,
                   const int32_t* tables, int32_t max_blocks, const int32_t* lens, int32_t batch,
@@ -64,6 +69,8 @@ struct DecodeArgs {
   size_t workspace_bytes;
   int32_t* dbg;
   cudaStream_t stream;
+  const float* k_scale = nullptr;  // E4M3 pools: row scales [num_blocks * Hkv * block_size]
+  const float* v_scale = nullptr;
 };
 
 size_t decode_workspace_size(int32_t batch, int32_t num_q_heads, const pkv_cache_desc& c);
@@ -98,6 +105,10 @@ int launch_prefill(const PrefillArgs& a);
 // [box_rows, 64]-element box and 128-byte swizzle. Returns false on failure.
 bool make_pool_tensor_map(void* map_out, const void* base, int64_t rows, int32_t head_dim,
                           int32_t box_rows);
+
+// Same over a pool of one-byte codes, box [box_rows, 128] (128-byte swizzle).
+bool make_pool_tensor_map_u8(void* map_out, const void* base, int64_t rows, int32_t head_dim,
+                             int32_t box_rows);
 
 // Encodes a bf16 tensor map of rank 1..5 with 128-byte swizzle; dims and
 // box innermost first, strides in bytes for dims 1..rank-1.

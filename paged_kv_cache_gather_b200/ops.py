@@ -16,7 +16,8 @@ import torch
 
 from . import _lib as L
 
-_DTYPES = {torch.float32: L.PKV_F32, torch.bfloat16: L.PKV_BF16}
+_DTYPES = {torch.float32: L.PKV_F32, torch.bfloat16: L.PKV_BF16, torch.uint8: L.PKV_FP8_E4M3,
+           torch.float8_e4m3fn: L.PKV_FP8_E4M3}
 
 
 @dataclass
@@ -143,6 +144,66 @@ def paged_kv_append(k, v, slot_mapping, k_cache, v_cache, dbg_err=None):
            "slot_mapping must be int64 [num_tokens] on the device")
     L.check(L.lib().paged_kv_append(_ptr(k), _ptr(v), _ptr(slot_mapping), T, _ptr(k_cache),
                                     _ptr(v_cache), cache_desc(k_cache), _ptr(dbg_err), _stream()))
+
+
+def _check_scales(k_scale, v_scale, k_cache):
+    nb, hkv, bs, _ = k_cache.shape
+    for t, name in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+        _check(t is not None and t.dtype == torch.float32 and t.device == k_cache.device and
+               t.is_contiguous() and t.numel() >= nb * hkv * bs,
+               f"{name} must be float32 [num_blocks, num_kv_heads, block_size] on the device")
+
+
+def paged_kv_append_fp8(k, v, slot_mapping, k_cache, v_cache, k_scale, v_scale, dbg_err=None):
+    """Quantise bf16 tokens into E4M3 pools (one float32 scale per stored row)."""
+    _check_pool(k_cache, v_cache)
+    _check(k_cache.dtype in (torch.uint8, torch.float8_e4m3fn), "pools must hold E4M3 codes")
+    _check_scales(k_scale, v_scale, k_cache)
+    dev = k_cache.device
+    T = k.shape[0]
+    _check(k.shape == (T, k_cache.shape[1], k_cache.shape[3]) and v.shape == k.shape and
+           k.dtype == torch.bfloat16 and v.dtype == torch.bfloat16 and k.is_contiguous() and
+           v.is_contiguous() and k.device == dev and v.device == dev,
+           "k, v must be contiguous bf16 [num_tokens, num_kv_heads, head_dim] on the device")
+    _check(slot_mapping.dtype == torch.int64 and slot_mapping.device == dev and
+           slot_mapping.numel() == T and slot_mapping.is_contiguous(),
+           "slot_mapping must be int64 [num_tokens] on the device")
+    L.check(L.lib().paged_kv_append_fp8(_ptr(k), _ptr(v), _ptr(slot_mapping), T, _ptr(k_cache),
+                                        _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+                                        cache_desc(k_cache), _ptr(dbg_err), _stream()))
+
+
+def paged_attention_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, block_tables, seq_lens,
+                               scale=None, mask_mod: Optional[MaskMod] = None, *, out=None,
+                               lse=None, workspace=None, dbg_err=None):
+    """Decode over E4M3 pools (bf16 q and out). Returns (out, lse)."""
+    _check_pool(k_cache, v_cache)
+    _check(k_cache.dtype in (torch.uint8, torch.float8_e4m3fn), "pools must hold E4M3 codes")
+    _check_scales(k_scale, v_scale, k_cache)
+    dev = k_cache.device
+    _i32(block_tables, "block_tables", dev)
+    _i32(seq_lens, "seq_lens", dev)
+    B, Hq, d = q.shape
+    _check(q.dtype == torch.bfloat16 and q.device == dev and q.is_contiguous(),
+           "q must be contiguous bf16 on the cache's device")
+    _check(d == k_cache.shape[3], "head_dim mismatch")
+    _check(block_tables.dim() == 2 and block_tables.shape[0] == B and seq_lens.numel() == B,
+           "block_tables [B, M] and seq_lens [B] must match q's batch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    mask_mod = mask_mod or no_mask()
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = decode_workspace(B, Hq, k_cache)
+    L.check(L.lib().paged_attention_decode_fp8(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), cache_desc(k_cache),
+        _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), B, Hq, float(scale),
+        mask_mod.to_c(B, dev, Hq), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _ptr(dbg_err), _stream()))
+    return out, lse
 
 
 def paged_kv_gather(k_cache, v_cache, block_tables, seq_lens, out_max_len, dbg_err=None):

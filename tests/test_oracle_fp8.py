@@ -63,3 +63,13 @@ def test_row_quantisation_error_bound_and_scale():
 def test_zero_row():
     codes, s = F.quantize_row(np.zeros(128, dtype=np.float32))
     assert s == 1.0 and not codes.any()
+
+
+def test_vectorised_rows_equal_row_by_row():
+    rng = np.random.default_rng(2)
+    x = (rng.normal(0, 1, (50, 128)) * rng.uniform(0.01, 100, (50, 1))).astype(np.float32)
+    x[3] = 0
+    codes, s = F.quantize_rows(x)
+    for i in range(50):
+        c1, s1 = F.quantize_row(x[i])
+        assert np.array_equal(codes[i], c1) and s[i] == s1
