@@ -211,6 +211,34 @@ class DecodeWork:
         self.h2d = (self.q_h[0].numel() * 2 + self.kn_h[0].numel() * 2 * 2 + B * 4 + B * 8
                     + self.tab_h.numel() * 4)
         self.d2h = self.out.numel() * 2 + self.lse.numel() * 4
+        # end-to-end steps: one host->device copy of every input of a step (packed
+        # into one pinned buffer per step) and one device->host copy of out + lse
+        parts = [("q", self.q_h[0]), ("kn", self.kn_h[0]), ("vn", self.vn_h[0]),
+                 ("lens", self.lens_h[0]), ("slots", self.slots_h[0]), ("tab", self.tab_h)]
+        self.layout, off = {}, 0
+        for name, t in parts:
+            nbytes = t.numel() * t.element_size()
+            self.layout[name] = (off, nbytes, t.dtype, tuple(t.shape))
+            off += (nbytes + 255) // 256 * 256
+        self.pack_h = torch.empty(steps, off, dtype=torch.uint8).pin_memory()
+        for st in range(steps):
+            for name, t in (("q", self.q_h[st]), ("kn", self.kn_h[st]), ("vn", self.vn_h[st]),
+                            ("lens", self.lens_h[st]), ("slots", self.slots_h[st]),
+                            ("tab", self.tab_h)):
+                o, nb, _, _ = self.layout[name]
+                self.pack_h[st, o:o + nb] = t.contiguous().view(torch.uint8).view(-1)
+        self.pack_d = torch.empty(off, dtype=torch.uint8, device=dev)
+        self.views = {name: self.pack_d[o:o + nb].view(dt).view(shape)
+                      for name, (o, nb, dt, shape) in self.layout.items()}
+        ob = self.out.numel() * 2
+        self.res_d = torch.empty((ob + 255) // 256 * 256 + self.lse.numel() * 4,
+                                 dtype=torch.uint8, device=dev)
+        self.res_h = torch.empty_like(self.res_d, device="cpu").pin_memory()
+        self.out_e = self.res_d[:ob].view(torch.bfloat16).view(B, Hq, D)
+        lo = (ob + 255) // 256 * 256
+        self.lse_e = self.res_d[lo:lo + self.lse.numel() * 4].view(torch.float32).view(B, Hq)
+        self.h2d = self.pack_h.shape[1]   # bytes actually copied per step (with alignment pads)
+        self.d2h = self.res_d.numel()
 
     def append(self, s):
         self.pkv.paged_kv_append(self.kn[s], self.vn[s], self.slots[s], self.k_cache, self.v_cache)
@@ -221,18 +249,13 @@ class DecodeWork:
                                         lse=self.lse, workspace=self.ws)
 
     def step_e2e(self, s, dev):
-        q = self.q_h[s].to(dev, non_blocking=True)
-        kn = self.kn_h[s].to(dev, non_blocking=True)
-        vn = self.vn_h[s].to(dev, non_blocking=True)
-        lens = self.lens_h[s].to(dev, non_blocking=True)
-        slots = self.slots_h[s].to(dev, non_blocking=True)
-        tab = self.tab_h.to(dev, non_blocking=True)
-        self.pkv.paged_kv_append(kn, vn, slots, self.k_cache, self.v_cache)
-        self.pkv.paged_attention_decode(q, self.k_cache, self.v_cache, tab, lens,
-                                        self.case.scale, self.mask, out=self.out, lse=self.lse,
-                                        workspace=self.ws)
-        self.out_h.copy_(self.out, non_blocking=True)
-        self.lse_h.copy_(self.lse, non_blocking=True)
+        self.pack_d.copy_(self.pack_h[s], non_blocking=True)
+        v = self.views
+        self.pkv.paged_kv_append(v["kn"], v["vn"], v["slots"], self.k_cache, self.v_cache)
+        self.pkv.paged_attention_decode(v["q"], self.k_cache, self.v_cache, v["tab"], v["lens"],
+                                        self.case.scale, self.mask, out=self.out_e,
+                                        lse=self.lse_e, workspace=self.ws)
+        self.res_h.copy_(self.res_d, non_blocking=True)
 
 
 class PrefillWork:
