@@ -58,12 +58,12 @@ def peaks():
 # after any change to them the bench reports null until they are profiled again.
 PROFILED_TRAFFIC = {
     "decode": {"sources": ['csrc/decode.cu', 'csrc/pkv_common.cuh'],
-               "sha256": "4dfba94f197e0cc5773e7e7c5c22ea82355203cedb893f59034d2023ef227efb",
-               "per_unit": 194786816 / 190134992,  # per algorithmic byte (16-seq ragged case)
+               "sha256": "d4dcc2488ce07563e9e3b74914303e3c9fbb2b94e2b63a8fe20394f10ba223eb",
+               "per_unit": 194071808 / 190134992,  # per algorithmic byte (16-seq ragged case)
                },
     "prefill": {"sources": ['csrc/prefill.cu', 'csrc/pkv_common.cuh', 'csrc/tc_sm100.cuh'],
-                "sha256": "d616477bd29b665cc799fcd7a0501dd3188c257a24e0f406fc4e586759a4cab6",
-                "per_unit": 299987200 / 1065168666624,  # per causal FLOP (1-seq case)
+                "sha256": "352d406ca921c1a65aeb530f16bd2fbb9fa7d45009559a1b45765f1950290cef",
+                "per_unit": 298716160 / 1065168666624,  # per causal FLOP (1-seq case)
                 },
 }
 
