@@ -508,7 +508,7 @@ def mask_modifiers(dev, d=None):
     return res
 
 
-def fp8_decode(dev, d):
+def fp8_decode(dev, d, n=20, warm=1):
     """The ragged decode batch on E4M3 pools: pools written by the quantising
     append from the bf16 pools, then decode timed (20 calls, inputs > L2).
     Reports the bytes read (codes + row scales) and the bf16-equivalent rate."""
@@ -534,8 +534,9 @@ def fp8_decode(dev, d):
     ws = pkv.decode_workspace(q.shape[0], q.shape[1], kc)
     call = lambda: pkv.paged_attention_decode_fp8(q, kc, vc, ks, vs, tab, lens, d.scale, mm,
                                                   out=o, lse=lse, workspace=ws)
-    call()
-    ms = time_calls(call, 20)
+    for _ in range(warm):
+        call()
+    ms = time_calls(call, n)
     vis = int(visible_tokens(d.seq_lens.numpy(), d.window_per_seq.numpy()).sum())
     fp8_bytes = vis * Hkv * 2 * (D + 4)
     bf16_bytes = vis * Hkv * 2 * D * 2
@@ -762,9 +763,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="all",
-                    choices=["all", "decode", "prefill", "shared_prefix"],
-                    help="shared_prefix: only the grouped decode of the beams workload "
-                         "(a side measurement, not the bench line)")
+                    choices=["all", "decode", "prefill", "shared_prefix", "fp8_decode"],
+                    help="shared_prefix / fp8_decode: only the grouped decode of the beams "
+                         "workload / the ragged decode on E4M3 pools (side measurements, not "
+                         "the bench line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the batch-1 sweep and the shared-prefix measurement")
@@ -782,6 +784,13 @@ def main():
     torch.cuda.set_device(dev)
     if args.workload == "shared_prefix":
         shared_prefix_only(args, dev, rank)
+        barrier(ws)
+        return
+    if args.workload == "fp8_decode":
+        from paged_kv_cache_gather_b200 import inputs as I
+        res = fp8_decode(dev, I.config3(), n=args.steps, warm=args.warmup)
+        if rank == 0:
+            print(json.dumps(res))
         barrier(ws)
         return
     pk, pk_kind = peaks()
