@@ -13,8 +13,10 @@ One step = one pass of the whole path over one batch of synthetic input:
 
 ``value`` is decode KV bytes per second (the metric's first part); the
 prefill half is reported in the ``prefill`` object. Inputs are resident in
-HBM when the device-timed region starts; ``e2e`` repeats the steps through
-the public API with pinned host buffers, copies inside the timed region.
+HBM when the device-timed region starts; ``e2e`` repeats the same interleaved
+steps through the public API with pinned host buffers: every step copies its
+inputs in and its results out inside the timed region, on side streams, so
+that a step's copies overlap the kernels next to it.
 
 ``--impl reference`` times the float64 CPU oracle (the only reference this
 method has) on a bounded sample of the same workload.
@@ -197,8 +199,6 @@ class DecodeWork:
         self.wps = c.window_per_seq.to(dev)
         self.out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
-        self.out_h = torch.empty_like(self.out, device="cpu").pin_memory()
-        self.lse_h = torch.empty_like(self.lse, device="cpu").pin_memory()
         import paged_kv_cache_gather_b200 as pkv
 
         self.pkv = pkv
@@ -208,9 +208,6 @@ class DecodeWork:
         self.kv_bytes = vis.sum(axis=1) * Hkv * D * 2 * 2  # K and V, bf16
         self.io_bytes = B * Hq * D * 2 * 2 + B * Hq * 4 + ((vis + 15) // 16).sum(1) * Hkv * 4
         self.append_bytes = B * Hkv * D * 2 * 2 * 2 + B * 8
-        self.h2d = (self.q_h[0].numel() * 2 + self.kn_h[0].numel() * 2 * 2 + B * 4 + B * 8
-                    + self.tab_h.numel() * 4)
-        self.d2h = self.out.numel() * 2 + self.lse.numel() * 4
         # end-to-end steps: one host->device copy of every input of a step (packed
         # into one pinned buffer per step) and one device->host copy of out + lse
         parts = [("q", self.q_h[0]), ("kn", self.kn_h[0]), ("vn", self.vn_h[0]),
@@ -227,18 +224,21 @@ class DecodeWork:
                             ("tab", self.tab_h)):
                 o, nb, _, _ = self.layout[name]
                 self.pack_h[st, o:o + nb] = t.contiguous().view(torch.uint8).view(-1)
-        self.pack_d = torch.empty(off, dtype=torch.uint8, device=dev)
-        self.views = {name: self.pack_d[o:o + nb].view(dt).view(shape)
-                      for name, (o, nb, dt, shape) in self.layout.items()}
+        # two device copies of the packed inputs and of the packed results, so
+        # that one step's copies overlap the neighbouring steps' kernels
+        self.pack_d = [torch.empty(off, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.views = [{name: pd[o:o + nb].view(dt).view(shape)
+                       for name, (o, nb, dt, shape) in self.layout.items()}
+                      for pd in self.pack_d]
         ob = self.out.numel() * 2
-        self.res_d = torch.empty((ob + 255) // 256 * 256 + self.lse.numel() * 4,
-                                 dtype=torch.uint8, device=dev)
-        self.res_h = torch.empty_like(self.res_d, device="cpu").pin_memory()
-        self.out_e = self.res_d[:ob].view(torch.bfloat16).view(B, Hq, D)
         lo = (ob + 255) // 256 * 256
-        self.lse_e = self.res_d[lo:lo + self.lse.numel() * 4].view(torch.float32).view(B, Hq)
+        rb = lo + self.lse.numel() * 4
+        self.res_d = [torch.empty(rb, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.res_h = [torch.empty(rb, dtype=torch.uint8).pin_memory() for _ in range(2)]
+        self.out_e = [r[:ob].view(torch.bfloat16).view(B, Hq, D) for r in self.res_d]
+        self.lse_e = [r[lo:rb].view(torch.float32).view(B, Hq) for r in self.res_d]
         self.h2d = self.pack_h.shape[1]   # bytes actually copied per step (with alignment pads)
-        self.d2h = self.res_d.numel()
+        self.d2h = rb
 
     def append(self, s):
         self.pkv.paged_kv_append(self.kn[s], self.vn[s], self.slots[s], self.k_cache, self.v_cache)
@@ -248,14 +248,19 @@ class DecodeWork:
                                         self.lens[s], self.case.scale, self.mask, out=self.out,
                                         lse=self.lse, workspace=self.ws)
 
-    def step_e2e(self, s, dev):
-        self.pack_d.copy_(self.pack_h[s], non_blocking=True)
-        v = self.views
+    # end-to-end step s through device buffer b: inputs in, kernels, results out
+    def e2e_in(self, s, b):
+        self.pack_d[b].copy_(self.pack_h[s], non_blocking=True)
+
+    def e2e_run(self, s, b):
+        v = self.views[b]
         self.pkv.paged_kv_append(v["kn"], v["vn"], v["slots"], self.k_cache, self.v_cache)
         self.pkv.paged_attention_decode(v["q"], self.k_cache, self.v_cache, v["tab"], v["lens"],
-                                        self.case.scale, self.mask, out=self.out_e,
-                                        lse=self.lse_e, workspace=self.ws)
-        self.res_h.copy_(self.res_d, non_blocking=True)
+                                        self.case.scale, self.mask, out=self.out_e[b],
+                                        lse=self.lse_e[b], workspace=self.ws)
+
+    def e2e_out(self, b):
+        self.res_h[b].copy_(self.res_d[b], non_blocking=True)
 
 
 class PrefillWork:
@@ -272,25 +277,42 @@ class PrefillWork:
         self.tab = c.block_tables.to(dev)
         self.ctx = c.ctx_lens.to(dev)
         self.ql = c.q_lens.to(dev)
-        self.q_h = c.q.pin_memory()
-        self.kn_h = c.k_new.pin_memory()
-        self.vn_h = c.v_new.pin_memory()
-        self.slots_h = c.slot_mapping.pin_memory()
-        self.q = self.q_h.to(dev)
-        self.kn = self.kn_h.to(dev)
-        self.vn = self.vn_h.to(dev)
-        self.slots = self.slots_h.to(dev)
+        self.q = c.q.to(dev)
+        self.kn = c.k_new.to(dev)
+        self.vn = c.v_new.to(dev)
+        self.slots = c.slot_mapping.to(dev)
         self.out = torch.empty_like(self.q)
         self.lse = torch.empty(self.q.shape[0], self.q.shape[1], dtype=torch.float32, device=dev)
-        self.out_h = torch.empty_like(self.out, device="cpu").pin_memory()
-        self.lse_h = torch.empty_like(self.lse, device="cpu").pin_memory()
         self.mask = pkv.causal()
+        # end-to-end steps: the inputs packed in one pinned host buffer (one
+        # host->device copy per step) and out + lse in one device->host copy;
+        # two device copies of each so that copies overlap the neighbouring steps
+        parts = [("q", c.q), ("kn", c.k_new), ("vn", c.v_new), ("slots", c.slot_mapping)]
+        layout, off = {}, 0
+        for name, t in parts:
+            nbytes = t.numel() * t.element_size()
+            layout[name] = (off, nbytes, t.dtype, tuple(t.shape))
+            off += (nbytes + 255) // 256 * 256
+        self.pack_h = torch.empty(off, dtype=torch.uint8).pin_memory()
+        for name, t in parts:
+            o, nb, _, _ = layout[name]
+            self.pack_h[o:o + nb] = t.contiguous().view(torch.uint8).view(-1)
+        self.pack_d = [torch.empty(off, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.views = [{name: pd[o:o + nb].view(dt).view(shape)
+                       for name, (o, nb, dt, shape) in layout.items()} for pd in self.pack_d]
+        ob = self.out.numel() * 2
+        lo = (ob + 255) // 256 * 256
+        rb = lo + self.lse.numel() * 4
+        self.res_d = [torch.empty(rb, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.res_h = [torch.empty(rb, dtype=torch.uint8).pin_memory() for _ in range(2)]
+        self.out_e = [r[:ob].view(torch.bfloat16).view(self.out.shape) for r in self.res_d]
+        self.lse_e = [r[lo:rb].view(torch.float32).view(self.lse.shape) for r in self.res_d]
         C = c.ctx_lens.numpy().astype(np.int64)
         Q = c.q_lens.numpy().astype(np.int64)
         pairs = (Q * C + Q * (Q + 1) // 2).sum()  # causally visible (query, key) pairs
         self.flops = float(4 * c.head_dim * pairs * c.num_q_heads)
-        self.h2d = (self.q.numel() + self.kn.numel() + self.vn.numel()) * 2 + self.slots.numel() * 8
-        self.d2h = self.out.numel() * 2 + self.lse.numel() * 4
+        self.h2d = off   # bytes actually copied per step (with alignment pads)
+        self.d2h = rb
 
     def append(self):
         self.pkv.paged_kv_append(self.kn, self.vn, self.slots, self.k_cache, self.v_cache)
@@ -300,16 +322,76 @@ class PrefillWork:
                                          self.tab, self.ctx, self.ql, self.mask,
                                          out=self.out, lse=self.lse)
 
-    def step_e2e(self, dev):
-        q = self.q_h.to(dev, non_blocking=True)
-        kn = self.kn_h.to(dev, non_blocking=True)
-        vn = self.vn_h.to(dev, non_blocking=True)
-        slots = self.slots_h.to(dev, non_blocking=True)
-        self.pkv.paged_kv_append(kn, vn, slots, self.k_cache, self.v_cache)
-        self.pkv.paged_attention_prefill(q, kn, vn, self.k_cache, self.v_cache, self.tab,
-                                         self.ctx, self.ql, self.mask, out=self.out, lse=self.lse)
-        self.out_h.copy_(self.out, non_blocking=True)
-        self.lse_h.copy_(self.lse, non_blocking=True)
+    def e2e_in(self, s, b):
+        self.pack_d[b].copy_(self.pack_h, non_blocking=True)
+
+    def e2e_run(self, s, b):
+        v = self.views[b]
+        self.pkv.paged_kv_append(v["kn"], v["vn"], v["slots"], self.k_cache, self.v_cache)
+        self.pkv.paged_attention_prefill(v["q"], v["kn"], v["vn"], self.k_cache, self.v_cache,
+                                         self.tab, self.ctx, self.ql, self.mask,
+                                         out=self.out_e[b], lse=self.lse_e[b])
+
+    def e2e_out(self, b):
+        self.res_h[b].copy_(self.res_d[b], non_blocking=True)
+
+
+def run_e2e(works, step_ids, stream):
+    """End-to-end steps through the public API, interleaved like the
+    device-timed steps (each step runs every work in `works` in turn). Every
+    work's step copies its inputs from pinned host memory to the device (one
+    copy), runs its kernels, and copies its results back (one copy). Copies run
+    on two side streams and step i uses device buffer i % 2, so the next
+    inputs arrive and the previous results leave while kernels run; events
+    order each buffer's reuse. Returns each work's device time in ms (CUDA
+    events on `stream`): from the point where the compute stream starts
+    waiting for that work's inputs to the end of its kernels, so a copy that
+    is not hidden is charged to its own work; the final copies out are charged
+    to the last work."""
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    tev = lambda: torch.cuda.Event(enable_timing=True)
+    K = len(works)
+    marks = []
+    h2d.wait_stream(stream)
+    d2h.wait_stream(stream)
+    ran = [[None, None] for _ in range(K)]
+    copied_in = [[None, None] for _ in range(K)]
+    copied_out = [[None, None] for _ in range(K)]
+    for i, s in enumerate(step_ids):
+        b = i % 2
+        for k, work in enumerate(works):
+            with torch.cuda.stream(h2d):
+                if ran[k][b] is not None:
+                    h2d.wait_event(ran[k][b])          # step i-2 no longer reads buffer b
+                work.e2e_in(s, b)
+                copied_in[k][b] = ev()
+                copied_in[k][b].record(h2d)
+            m = tev()
+            m.record(stream)
+            marks.append((k, m))
+            stream.wait_event(copied_in[k][b])
+            if copied_out[k][b] is not None:
+                stream.wait_event(copied_out[k][b])    # step i-2's results have left buffer b
+            with torch.cuda.stream(stream):
+                work.e2e_run(s, b)
+            ran[k][b] = ev()
+            ran[k][b].record(stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(ran[k][b])
+                work.e2e_out(b)
+                copied_out[k][b] = ev()
+                copied_out[k][b].record(d2h)
+    stream.wait_stream(h2d)
+    stream.wait_stream(d2h)
+    end = tev()
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = [0.0] * K
+    for j, (k, m) in enumerate(marks):
+        nxt = marks[j + 1][1] if j + 1 < len(marks) else end
+        ms[k] += m.elapsed_time(nxt)
+    return ms
 
 
 # ------------------------------------------------------------------ side measurements
@@ -855,22 +937,13 @@ def main():
     ms_total = max_over_ranks(t_start.elapsed_time(t_end), ws, dev)
 
     # ---------------- end-to-end region (host buffers, copies inside)
-    e2e_steps = n
+    step_ids = list(range(args.warmup, args.warmup + n))
     torch.cuda.synchronize()
     barrier(ws)
-    e_start, e_end, e_mid = ev(), ev(), [ev() for _ in range(e2e_steps)]
-    e_pre = [ev() for _ in range(e2e_steps)]
-    e_start.record(stream)
-    for i in range(e2e_steps):
-        s = args.warmup + i
-        e_pre[i].record(stream)
-        if dw:
-            dw.step_e2e(s, dev)
-        e_mid[i].record(stream)
-        if pw:
-            pw.step_e2e(dev)
-    e_end.record(stream)
-    torch.cuda.synchronize()
+    works = [w for w in (dw, pw) if w is not None]
+    e2e_ms_list = run_e2e(works, step_ids, stream)
+    e2e_dec_ms = e2e_ms_list[0] if dw else None
+    e2e_pre_ms = e2e_ms_list[-1] if pw else None
     barrier(ws)
     clk = clocks.stop()
 
@@ -889,8 +962,7 @@ def main():
         # whole-job KV throughput of the decode steps (append + decode), all ranks
         value = kv * ws / (dec_total_ms * 1e-3) / 1e9
         achieved = (kv + io) / n / (dec_only_ms / n * 1e-3) / 1e9
-        e2e_ms = sum(e_pre[i].elapsed_time(e_mid[i]) for i in range(e2e_steps))
-        e2e_ms = max_over_ranks(e2e_ms, ws, dev)
+        e2e_ms = max_over_ranks(e2e_dec_ms, ws, dev)
         line.update({
             "value": round(value, 2), "unit": "GB/s",
             "decode": {"ms_per_step": round(dec_total_ms / n, 4),
@@ -914,9 +986,7 @@ def main():
         pre_ms_t = max_over_ranks(sum(pre_ms), ws, dev)
         pstep_ms = max_over_ranks(sum(pre_ms) + sum(papp_ms), ws, dev)
         tf = pw.flops * n / (pre_ms_t * 1e-3) / 1e12
-        pe2e = sum(e_mid[i].elapsed_time(e_pre[i + 1] if i + 1 < e2e_steps else e_end)
-                   for i in range(e2e_steps))
-        pe2e = max_over_ranks(pe2e, ws, dev)
+        pe2e = max_over_ranks(e2e_pre_ms, ws, dev)
         peak_tf = pk["bf16_tflops"]
         line["prefill"] = {
             "value": round(pw.flops * n * ws / (pstep_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
