@@ -56,29 +56,42 @@ def peaks():
 
 # DRAM bytes (read + write) per unit of work, from one ncu capture of each
 # kernel on a smaller case of the same workload (profiles/*.md); a full launch
-# scales it by its units. Valid only for the kernel sources it was taken on:
-# after any change to them the bench reports null until they are profiled again.
+# scales it by its units. Valid only for the kernel code it was taken on: after
+# any change to that code (comments aside) the bench reports null until the
+# kernels are profiled again.
 PROFILED_TRAFFIC = {
     "decode": {"sources": ['csrc/decode.cu', 'csrc/pkv_common.cuh'],
-               "sha256": "d4dcc2488ce07563e9e3b74914303e3c9fbb2b94e2b63a8fe20394f10ba223eb",
+               "code_sha256": "f87eca92834f355213fdd1e53f086b5fa3bb0f33c46c8ad5180dda7d33d415b3",
                "per_unit": 194071808 / 190134992,  # per algorithmic byte (16-seq ragged case)
                },
     "prefill": {"sources": ['csrc/prefill.cu', 'csrc/pkv_common.cuh', 'csrc/tc_sm100.cuh'],
-                "sha256": "352d406ca921c1a65aeb530f16bd2fbb9fa7d45009559a1b45765f1950290cef",
+                "code_sha256": "b082f2e11624b3fc4976dd311201411e6ae21473f26a430a7fe378f8cd6012a8",
                 "per_unit": 298716160 / 1065168666624,  # per causal FLOP (1-seq case)
                 },
 }
 
 
-def profiled_traffic(kind, units):
+def code_hash(sources):
+    """sha256 of the kernel sources with comments and blank lines removed, so
+    that an edit of a comment keeps the recorded counters while any change of
+    code drops them (the sources hold no comment markers inside strings)."""
     import hashlib
+    import re
 
-    rec = PROFILED_TRAFFIC[kind]
     h = hashlib.sha256()
-    for f in rec["sources"]:
-        with open(os.path.join(ROOT, "paged_kv_cache_gather_b200", f), "rb") as fh:
-            h.update(fh.read())
-    if h.hexdigest() != rec["sha256"]:
+    for f in sources:
+        with open(os.path.join(ROOT, "paged_kv_cache_gather_b200", f)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        lines = [ln.rstrip() for ln in text.splitlines() if ln.strip()]
+        h.update("\n".join(lines).encode())
+    return h.hexdigest()
+
+
+def profiled_traffic(kind, units):
+    rec = PROFILED_TRAFFIC[kind]
+    if code_hash(rec["sources"]) != rec["code_sha256"]:
         return None
     return int(rec["per_unit"] * units)
 

@@ -419,11 +419,23 @@ PKV_API int paged_attention_decode_noalloc(const void* q, const void* k_cache, c
 
 /*
  * pkv_debug_exp2 — diagnostic, not part of the attention API: y[i] = 2^x[i]
- * computed by the FMA-pipe exponential the prefill softmax uses for part of its
- * elements (exact base-2 range reduction plus a fitted cubic; relative error
- * <= 1e-4 for -126 <= x <= 127, exactly 0 below -126). x, y: device float32 [n].
+ * computed by the library's FMA-pipe exponential (exact base-2 range reduction
+ * plus a fitted cubic; relative error <= 1e-4 for -126 <= x <= 127, exactly 0
+ * below -126), a building block for taking exponentials off the MUFU unit that
+ * the attention kernels do not use at present. x, y: device float32 [n].
  */
 PKV_API int pkv_debug_exp2(const float* x, float* y, int32_t n, void* stream);
+
+/*
+ * pkv_debug_wait_timeout — diagnostic, not part of the attention API: one warp
+ * waits on a shared-memory mbarrier that nothing arrives on, through the
+ * library's bounded wait (the one every TMA/MMA wait in the kernels uses). When
+ * the wait gives up (after about 4 s) the kernel sets PKV_DBG_TIMEOUT in
+ * *dbg_err and returns; the context stays usable. elapsed_ns (device, nullable)
+ * receives the globaltimer nanoseconds the wait took. It exists so that the
+ * timeout path can be tested without a stuck copy or any GPU fault.
+ */
+PKV_API int pkv_debug_wait_timeout(int32_t* dbg_err, uint64_t* elapsed_ns, void* stream);
 
 /* Name of a status code (static string). */
 PKV_API const char* pkv_status_string(int status);

@@ -57,6 +57,7 @@ EXPORTS = (
     "paged_kv_append_fp8",
     "paged_attention_decode_fp8",
     "pkv_debug_exp2",
+    "pkv_debug_wait_timeout",
     "pkv_status_string",
     "pkv_last_error",
     "pkv_version",
@@ -134,6 +135,8 @@ def _declare(lib):
     lib.paged_attention_decode_fp8.restype = ctypes.c_int
     lib.pkv_debug_exp2.argtypes = [_vp, _vp, _i32, _vp]
     lib.pkv_debug_exp2.restype = ctypes.c_int
+    lib.pkv_debug_wait_timeout.argtypes = [_vp, _vp, _vp]
+    lib.pkv_debug_wait_timeout.restype = ctypes.c_int
     lib.pkv_status_string.argtypes = [ctypes.c_int]
     lib.pkv_status_string.restype = ctypes.c_char_p
     lib.pkv_last_error.argtypes = []

@@ -342,4 +342,31 @@ int pkv_debug_exp2(const float* x, float* y, int32_t n, void* stream) {
   return check_launch("pkv_debug_exp2");
 }
 
+// One warp waits on an mbarrier that nothing arrives on, through the same
+// bounded wait every kernel of the library uses (bursts of try_wait, a
+// globaltimer check between bursts, 4 s limit); when the wait gives up it sets
+// PKV_DBG_TIMEOUT and the kernel returns normally.
+__global__ void __launch_bounds__(32) debug_wait_timeout_kernel(int32_t* dbg, uint64_t* elapsed_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  const uint64_t t0 = global_ns();
+  const bool ok = mbar_wait(smem_u32(&bar), 0);
+  const uint64_t t1 = global_ns();
+  if (threadIdx.x == 0) {
+    if (!ok) flag_error(dbg, PKV_DBG_TIMEOUT);
+    if (elapsed_ns) *elapsed_ns = t1 - t0;
+  }
+}
+
+int pkv_debug_wait_timeout(int32_t* dbg_err, uint64_t* elapsed_ns, void* stream) {
+  g_last_error[0] = 0;
+  if (!dbg_err) return fail(PKV_ERR_INVALID_ARG, "pkv_debug_wait_timeout: null debug word");
+  debug_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(dbg_err, elapsed_ns);
+  return check_launch("pkv_debug_wait_timeout");
+}
+
 }  // extern "C"

@@ -214,8 +214,9 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x on the FMA pipe, for x <= 127 (used for part of the softmax exponentials
-// so the MUFU unit is not the only one doing them). Exact base-2 range
+// 2^x on the FMA pipe, for x <= 127: a building block for moving part of a
+// softmax's exponentials off the MUFU unit (the prefill kernel measured slower
+// with it on 1/16 to 1/4 of its elements, so it does not use it). Exact base-2 range
 // reduction x = j + f, j = round(x) (via the 1.5*2^23 rounding constant),
 // f in [-1/2, 1/2]; 2^f by a cubic fitted for minimum relative error
 // (paged_kv_cache_gather_b200/fit_exp2.py: max relative error 7.5e-5, 1.0e-4

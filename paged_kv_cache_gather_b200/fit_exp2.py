@@ -1,4 +1,5 @@
-"""Fit the polynomial behind the FMA-pipe exp2 of the prefill softmax.
+"""Fit the polynomial behind the library's FMA-pipe exp2 (a building block for
+taking softmax exponentials off the MUFU unit).
 
 2^x is split exactly (Cody and Waite's range reduction, here in base 2 where it
 is exact): x = j + f with j = round(x) and f in [-1/2, 1/2], so

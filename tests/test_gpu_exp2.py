@@ -1,6 +1,7 @@
-"""GPU: the FMA-pipe exponential used for part of the prefill softmax against
-exp2 in float64: relative error <= 2e-4 on [-126, 8.5] (the kernel only feeds
-it values <= 8), exactly 0 below -126 and for -inf."""
+"""GPU: the library's FMA-pipe exponential (a building block for taking softmax
+exponentials off the MUFU unit) against exp2 in float64: relative error <= 2e-4
+on [-126, 8.5] (a softmax with a lazy maximum feeds it values <= 8), exactly 0
+below -126 and for -inf."""
 
 import ctypes
 
