@@ -25,7 +25,9 @@ Pins (see ``tests/test_oracle_pins.py``): dense attention from a different
 library routine on a contiguous layout, invariance under permutation of the
 physical blocks, closed forms (identical keys, a dominant key, W >= L), a
 pure-Python brute force on tiny inputs, split-and-merge of the softmax, and
-shared-vs-copied prefixes. No function here is parity-unpinned.
+shared-vs-copied prefixes; ``tests/test_golden.py`` checks decode, prefill,
+append and gather against a worked example with hand-derived exact answers
+(``tests/golden/``). No function here is parity-unpinned.
 """
 
 from .attention64 import (  # noqa: F401
