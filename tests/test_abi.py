@@ -121,3 +121,105 @@ def test_workspace_size_is_zero_for_fp32_and_positive_for_bf16(lib):
     assert lib.paged_attention_decode_workspace_size(4, 8, desc(dt=L.PKV_F32, d=64)) == 0
     assert lib.paged_attention_decode_workspace_size(4, 8, desc()) > 0
     assert lib.paged_attention_decode_workspace_size(4, 7, desc()) == 0
+
+
+E4M3 = getattr(L, "PKV_FP8_E4M3", 2)
+
+
+def test_fp8_argument_checks(lib):
+    fp8 = desc(dt=E4M3)
+
+    def dec(c=fp8, ks=FAKE, vs=FAKE, **kw):
+        a = dict(B=2, Hq=8, out=FAKE, m=mask())
+        a.update(kw)
+        return lib.paged_attention_decode_fp8(FAKE, FAKE, FAKE, ks, vs, c, FAKE, 4, FAKE, a["B"],
+                                              a["Hq"], 0.1, a["m"], a["out"], FAKE, FAKE,
+                                              1 << 30, None, None)
+    assert dec(c=desc()) == L.PKV_ERR_INVALID_ARG            # not an E4M3 pool
+    assert dec(ks=None) == L.PKV_ERR_INVALID_ARG             # E4M3 needs the row scales
+    assert dec(out=None) == L.PKV_ERR_INVALID_ARG
+    assert dec(Hq=7) == L.PKV_ERR_INVALID_ARG
+    assert dec(B=0) == L.PKV_OK
+    # plain decode refuses row scales; the E4M3 append refuses other pools
+    st = lib.paged_attention_decode(FAKE, FAKE, FAKE, fp8, FAKE, 4, FAKE, 2, 8, 0.1, mask(),
+                                    FAKE, FAKE, FAKE, 1 << 30, None, None)
+    assert st == L.PKV_ERR_INVALID_ARG
+    assert lib.paged_kv_append_fp8(FAKE, FAKE, FAKE, 2, FAKE, FAKE, FAKE, FAKE, desc(), None,
+                                   None) == L.PKV_ERR_UNSUPPORTED
+    assert lib.paged_kv_append_fp8(FAKE, FAKE, FAKE, 2, FAKE, FAKE, FAKE, FAKE,
+                                   desc(dt=E4M3, d=64), None, None) == L.PKV_ERR_UNSUPPORTED
+    assert lib.paged_kv_append_fp8(FAKE, FAKE, FAKE, 2, FAKE, FAKE, None, FAKE, fp8, None,
+                                   None) == L.PKV_ERR_INVALID_ARG
+    assert lib.paged_kv_append_fp8(FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, fp8, None,
+                                   None) == L.PKV_OK
+    # E4M3 pools are refused where their row scales would have to move
+    assert lib.paged_kv_append(FAKE, FAKE, FAKE, 2, FAKE, FAKE, fp8, None,
+                               None) == L.PKV_ERR_UNSUPPORTED
+    assert lib.paged_kv_copy_blocks(FAKE, FAKE, fp8, FAKE, 1, None,
+                                    None) == L.PKV_ERR_UNSUPPORTED
+
+
+def test_copy_blocks_argument_checks(lib):
+    assert lib.paged_kv_copy_blocks(FAKE, FAKE, desc(), FAKE, -1, None,
+                                    None) == L.PKV_ERR_INVALID_ARG
+    assert lib.paged_kv_copy_blocks(FAKE, FAKE, desc(), None, 2, None,
+                                    None) == L.PKV_ERR_INVALID_ARG
+    assert lib.paged_kv_copy_blocks(ctypes.c_void_p(0x10004), FAKE, desc(), FAKE, 2, None,
+                                    None) == L.PKV_ERR_INVALID_ARG
+    assert lib.paged_kv_copy_blocks(FAKE, FAKE, desc(), FAKE, 0, None, None) == L.PKV_OK
+
+
+def test_shared_prefix_argument_checks(lib):
+    def call(c=None, m=None, **kw):
+        a = dict(B=8, Hq=16, groups=2, gmax=4, out=FAKE, scale=0.1, ws=1 << 30)
+        a.update(kw)
+        return lib.paged_attention_decode_shared_prefix(
+            FAKE, FAKE, FAKE, c or desc(), FAKE, 4, FAKE, a["B"], a["Hq"], a["scale"],
+            m or mask(1), FAKE, a["groups"], a["gmax"], FAKE, a["out"], FAKE, FAKE, a["ws"],
+            None, None)
+    assert call(c=desc(d=64)) == L.PKV_ERR_UNSUPPORTED         # bf16, head_dim 128 only
+    assert call(c=desc(bs=4)) == L.PKV_ERR_UNSUPPORTED         # block_size >= 8
+    assert call(m=mask(2, 64)) == L.PKV_ERR_UNSUPPORTED        # no sliding window
+    assert call(Hq=7) == L.PKV_ERR_INVALID_ARG
+    assert call(Hq=2 * 33) == L.PKV_ERR_UNSUPPORTED            # > 32 query heads per KV head
+    assert call(scale=float("nan")) == L.PKV_ERR_INVALID_ARG
+    assert call(groups=0) == L.PKV_ERR_INVALID_ARG
+    assert call(groups=9) == L.PKV_ERR_INVALID_ARG             # more groups than sequences
+    assert call(Hq=2 * 32, gmax=8) == L.PKV_ERR_UNSUPPORTED    # group rows beyond 128
+    assert call(out=None) == L.PKV_ERR_INVALID_ARG
+    assert call(ws=16) == L.PKV_ERR_WORKSPACE_TOO_SMALL
+    assert call(B=0) == L.PKV_OK
+    assert lib.paged_attention_decode_shared_prefix_workspace_size(8, 16, desc()) > 0
+
+
+def test_block_mask_and_reserve_argument_checks(lib):
+    def bm(**kw):
+        a = dict(B=2, Hq=8, qt=128, kt=128, nq=4, nk=4, out=FAKE, m=mask(1))
+        a.update(kw)
+        return lib.paged_attention_block_mask(FAKE, FAKE, a["B"], a["Hq"], a["m"], a["qt"],
+                                              a["kt"], a["nq"], a["nk"], a["out"], None)
+    assert bm(qt=0) == L.PKV_ERR_INVALID_ARG
+    assert bm(B=-1) == L.PKV_ERR_INVALID_ARG
+    assert bm(out=None) == L.PKV_ERR_INVALID_ARG
+    assert bm(m=mask(7)) == L.PKV_ERR_INVALID_ARG
+    assert bm(nq=0) == L.PKV_OK
+
+    def rs(c=None, **kw):
+        a = dict(B=4, T=4, mb=8, stack=FAKE)
+        a.update(kw)
+        return lib.paged_kv_reserve_slots(FAKE, FAKE, c or desc(), FAKE, a["mb"], FAKE, FAKE,
+                                          a["B"], a["stack"], FAKE, FAKE, FAKE, FAKE, a["T"],
+                                          FAKE, None, None)
+    assert rs(c=desc(dt=E4M3)) == L.PKV_ERR_UNSUPPORTED
+    assert rs(T=-1) == L.PKV_ERR_INVALID_ARG
+    assert rs(mb=0) == L.PKV_ERR_INVALID_ARG
+    assert rs(B=8193) == L.PKV_ERR_UNSUPPORTED
+    assert rs(stack=None) == L.PKV_ERR_INVALID_ARG
+    assert rs(B=0) == L.PKV_OK
+    assert lib.paged_kv_reserve_scratch_size(desc()) > 0
+
+
+def test_debug_entries_reject_bad_arguments(lib):
+    assert lib.pkv_debug_exp2(FAKE, FAKE, -1, None) == L.PKV_ERR_INVALID_ARG
+    assert lib.pkv_debug_exp2(FAKE, FAKE, 0, None) == L.PKV_OK
+    assert lib.pkv_debug_wait_timeout(None, None, None) == L.PKV_ERR_INVALID_ARG
