@@ -192,6 +192,19 @@ PKV_API int paged_kv_copy_blocks(void* k_cache, void* v_cache, pkv_cache_desc ca
                                  int32_t* dbg_err, void* stream);
 
 /*
+ * paged_kv_copy_blocks_fp8 — paged_kv_copy_blocks for E4M3 pools: each pair
+ * copies block src's codes (K and V) and its row scales (k_scale, v_scale:
+ * float32 [num_blocks, num_kv_heads, block_size], 16-byte aligned) to block
+ * dst, so a copied row decodes to the same values. Requires
+ * num_kv_heads * block_size to be a multiple of 4; same pair rules and error
+ * reporting as paged_kv_copy_blocks. Two kernel launches on `stream`.
+ */
+PKV_API int paged_kv_copy_blocks_fp8(void* k_cache, void* v_cache, float* k_scale,
+                                     float* v_scale, pkv_cache_desc cache,
+                                     const int32_t* block_pairs, int32_t num_pairs,
+                                     int32_t* dbg_err, void* stream);
+
+/*
  * paged_kv_reserve_slots — device-side block allocation for an append step:
  * slots for the new tokens, new blocks from a free stack, copy-on-write of
  * shared partly filled blocks; no host round trip (CUDA-graph capturable).
@@ -228,6 +241,20 @@ PKV_API int paged_kv_copy_blocks(void* k_cache, void* v_cache, pkv_cache_desc ca
  * Three kernel launches on `stream`.
  */
 PKV_API size_t paged_kv_reserve_scratch_size(pkv_cache_desc cache);
+/*
+ * paged_kv_reserve_slots_fp8 — paged_kv_reserve_slots for E4M3 pools: the
+ * same bookkeeping, and each copy-on-write also copies the block's row scales
+ * (k_scale, v_scale as in paged_kv_copy_blocks_fp8). paged_kv_reserve_slots
+ * rejects E4M3 pools. Four kernel launches on `stream`.
+ */
+PKV_API int paged_kv_reserve_slots_fp8(void* k_cache, void* v_cache, float* k_scale,
+                                       float* v_scale, pkv_cache_desc cache,
+                                       int32_t* block_tables, int32_t max_blocks_per_seq,
+                                       int32_t* seq_lens, const int32_t* num_new, int32_t batch,
+                                       int32_t* free_stack, int32_t* free_top, int32_t* refcount,
+                                       int32_t* scratch, int64_t* slot_mapping,
+                                       int32_t num_tokens, int32_t* cow_pairs, int32_t* dbg_err,
+                                       void* stream);
 PKV_API int paged_kv_reserve_slots(void* k_cache, void* v_cache, pkv_cache_desc cache,
                                    int32_t* block_tables, int32_t max_blocks_per_seq,
                                    int32_t* seq_lens, const int32_t* num_new, int32_t batch,

@@ -6,8 +6,10 @@ Calls (thin bindings over the C ABI in ``include/pagedkv.h``):
 * ``paged_kv_gather``         block tables resolved to contiguous K/V
 * ``paged_kv_append_fp8`` / ``paged_attention_decode_fp8``  E4M3 pools with
   per-row scales (half the bytes per token)
-* ``paged_kv_copy_blocks``    copy-on-write of shared blocks
-* ``paged_kv_reserve_slots``  device-side block allocation (growth + copy-on-write)
+* ``paged_kv_copy_blocks``    copy-on-write of shared blocks (``_fp8``: E4M3
+  pools, row scales copied with the codes)
+* ``paged_kv_reserve_slots``  device-side block allocation (growth + copy-on-write;
+  E4M3 pools pass their row scales)
 * ``paged_attention_decode``  one query per sequence over paged KV
 * ``paged_attention_prefill`` a chunk of queries over paged context + chunk
 * ``paged_attention_decode_shared_prefix``  decode for groups (beams,
@@ -35,6 +37,7 @@ from .ops import (  # noqa: F401
     paged_kv_append,
     paged_kv_append_fp8,
     paged_kv_copy_blocks,
+    paged_kv_copy_blocks_fp8,
     paged_kv_gather,
     paged_kv_reserve_slots,
     prefix_lm,

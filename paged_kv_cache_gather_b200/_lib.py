@@ -45,6 +45,7 @@ EXPORTS = (
     "paged_kv_append",
     "paged_kv_gather",
     "paged_kv_copy_blocks",
+    "paged_kv_copy_blocks_fp8",
     "paged_attention_decode_workspace_size",
     "paged_attention_decode",
     "paged_attention_prefill",
@@ -54,6 +55,7 @@ EXPORTS = (
     "paged_attention_block_mask",
     "paged_kv_reserve_scratch_size",
     "paged_kv_reserve_slots",
+    "paged_kv_reserve_slots_fp8",
     "paged_kv_append_fp8",
     "paged_attention_decode_fp8",
     "pkv_debug_exp2",
@@ -100,6 +102,8 @@ def _declare(lib):
     lib.paged_kv_gather.restype = ctypes.c_int
     lib.paged_kv_copy_blocks.argtypes = [_vp, _vp, CacheDescC, _vp, _i32, _vp, _vp]
     lib.paged_kv_copy_blocks.restype = ctypes.c_int
+    lib.paged_kv_copy_blocks_fp8.argtypes = [_vp, _vp, _vp, _vp, CacheDescC, _vp, _i32, _vp, _vp]
+    lib.paged_kv_copy_blocks_fp8.restype = ctypes.c_int
     lib.paged_attention_decode_workspace_size.argtypes = [_i32, _i32, CacheDescC]
     lib.paged_attention_decode_workspace_size.restype = _sz
     lib.paged_attention_decode.argtypes = [_vp, _vp, _vp, CacheDescC, _vp, _i32, _vp, _i32, _i32,
@@ -126,6 +130,10 @@ def _declare(lib):
     lib.paged_kv_reserve_slots.argtypes = [_vp, _vp, CacheDescC, _vp, _i32, _vp, _vp, _i32, _vp,
                                            _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp]
     lib.paged_kv_reserve_slots.restype = ctypes.c_int
+    lib.paged_kv_reserve_slots_fp8.argtypes = [_vp, _vp, _vp, _vp, CacheDescC, _vp, _i32, _vp,
+                                               _vp, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp,
+                                               _vp, _vp]
+    lib.paged_kv_reserve_slots_fp8.restype = ctypes.c_int
     lib.paged_kv_append_fp8.argtypes = [_vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, CacheDescC, _vp,
                                         _vp]
     lib.paged_kv_append_fp8.restype = ctypes.c_int

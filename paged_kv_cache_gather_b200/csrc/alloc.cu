@@ -248,26 +248,35 @@ PKV_API size_t paged_kv_reserve_scratch_size(pkv_cache_desc cache) {
   return (size_t)2 * cache.num_blocks * sizeof(int32_t);
 }
 
-PKV_API int paged_kv_reserve_slots(void* k_cache, void* v_cache, pkv_cache_desc cache,
-                                   int32_t* block_tables, int32_t max_blocks_per_seq,
-                                   int32_t* seq_lens, const int32_t* num_new, int32_t batch,
-                                   int32_t* free_stack, int32_t* free_top, int32_t* refcount,
-                                   int32_t* scratch, int64_t* slot_mapping, int32_t num_tokens,
-                                   int32_t* cow_pairs, int32_t* dbg_err, void* stream) {
-  const char* fn = "paged_kv_reserve_slots";
+// The reserve step; k_scale / v_scale are the row scales of E4M3 pools (copied
+// with the codes), null for other pools.
+static int reserve(const char* fn, void* k_cache, void* v_cache, float* k_scale, float* v_scale,
+                   pkv_cache_desc cache, int32_t* block_tables, int32_t max_blocks_per_seq,
+                   int32_t* seq_lens, const int32_t* num_new, int32_t batch, int32_t* free_stack,
+                   int32_t* free_top, int32_t* refcount, int32_t* scratch,
+                   int64_t* slot_mapping, int32_t num_tokens, int32_t* cow_pairs,
+                   int32_t* dbg_err, void* stream) {
   clear_last_error();
   if (int st = check_cache(cache, fn)) return st;
-  if (cache.dtype == PKV_FP8_E4M3)
-    return fail(PKV_ERR_UNSUPPORTED, "%s: E4M3 pools (row scales) not supported", fn);
+  const bool fp8 = cache.dtype == PKV_FP8_E4M3;
+  if (fp8 != (k_scale != nullptr))
+    return fail(PKV_ERR_UNSUPPORTED, "%s: %s", fn,
+                fp8 ? "E4M3 pools take paged_kv_reserve_slots_fp8 (row scales move with blocks)"
+                    : "row scales belong to E4M3 pools");
+  const int64_t scale_bytes = (int64_t)cache.num_kv_heads * cache.block_size * 4;
+  if (fp8 && scale_bytes % 16)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: num_kv_heads * block_size must be a multiple of 4", fn);
   if (batch < 0 || num_tokens < 0 || max_blocks_per_seq <= 0)
     return fail(PKV_ERR_INVALID_ARG, "%s: bad batch, num_tokens or max_blocks_per_seq", fn);
   if (batch > kMaxReserveBatch)
     return fail(PKV_ERR_UNSUPPORTED, "%s: batch %d > %d", fn, batch, kMaxReserveBatch);
   if (batch == 0) return PKV_OK;
   if (!k_cache || !v_cache || !block_tables || !seq_lens || !num_new || !free_stack ||
-      !free_top || !refcount || !scratch || (num_tokens > 0 && !slot_mapping) || !cow_pairs)
+      !free_top || !refcount || !scratch || (num_tokens > 0 && !slot_mapping) || !cow_pairs ||
+      (fp8 && !v_scale))
     return fail(PKV_ERR_INVALID_ARG, "%s: null pointer", fn);
-  if (!aligned16(k_cache) || !aligned16(v_cache))
+  if (!aligned16(k_cache) || !aligned16(v_cache) ||
+      (fp8 && (!aligned16(k_scale) || !aligned16(v_scale))))
     return fail(PKV_ERR_INVALID_ARG, "%s: pools must be 16-byte aligned", fn);
   ReserveParams p = {};
   p.tables = block_tables;
@@ -303,7 +312,42 @@ PKV_API int paged_kv_reserve_slots(void* k_cache, void* v_cache, pkv_cache_desc 
   }
   reserve_apply_kernel<<<1, kThreads, smem, s>>>(p);
   if (int st = check_launch(fn)) return st;
-  return launch_copy_blocks(k_cache, v_cache, cache, cow_pairs, batch, dbg_err, s, true);
+  if (int st = launch_copy_blocks(k_cache, v_cache, cache, cow_pairs, batch, dbg_err, s, true))
+    return st;
+  if (!fp8) return PKV_OK;
+  return launch_copy_spans(k_scale, v_scale, scale_bytes, cache.num_blocks, cow_pairs, batch,
+                           dbg_err, s, true);
+}
+
+PKV_API int paged_kv_reserve_slots(void* k_cache, void* v_cache, pkv_cache_desc cache,
+                                   int32_t* block_tables, int32_t max_blocks_per_seq,
+                                   int32_t* seq_lens, const int32_t* num_new, int32_t batch,
+                                   int32_t* free_stack, int32_t* free_top, int32_t* refcount,
+                                   int32_t* scratch, int64_t* slot_mapping, int32_t num_tokens,
+                                   int32_t* cow_pairs, int32_t* dbg_err, void* stream) {
+  return reserve("paged_kv_reserve_slots", k_cache, v_cache, nullptr, nullptr, cache,
+                 block_tables, max_blocks_per_seq, seq_lens, num_new, batch, free_stack,
+                 free_top, refcount, scratch, slot_mapping, num_tokens, cow_pairs, dbg_err,
+                 stream);
+}
+
+PKV_API int paged_kv_reserve_slots_fp8(void* k_cache, void* v_cache, float* k_scale,
+                                       float* v_scale, pkv_cache_desc cache,
+                                       int32_t* block_tables, int32_t max_blocks_per_seq,
+                                       int32_t* seq_lens, const int32_t* num_new, int32_t batch,
+                                       int32_t* free_stack, int32_t* free_top, int32_t* refcount,
+                                       int32_t* scratch, int64_t* slot_mapping,
+                                       int32_t num_tokens, int32_t* cow_pairs, int32_t* dbg_err,
+                                       void* stream) {
+  const char* fn = "paged_kv_reserve_slots_fp8";
+  if (cache.dtype != PKV_FP8_E4M3 || !k_scale) {
+    clear_last_error();
+    return fail(cache.dtype != PKV_FP8_E4M3 ? PKV_ERR_UNSUPPORTED : PKV_ERR_INVALID_ARG,
+                "%s: E4M3 pools with their row scales only", fn);
+  }
+  return reserve(fn, k_cache, v_cache, k_scale, v_scale, cache, block_tables,
+                 max_blocks_per_seq, seq_lens, num_new, batch, free_stack, free_top, refcount,
+                 scratch, slot_mapping, num_tokens, cow_pairs, dbg_err, stream);
 }
 
 }  // extern "C"

@@ -207,6 +207,30 @@ int paged_kv_copy_blocks(void* k_cache, void* v_cache, pkv_cache_desc cache,
                             static_cast<cudaStream_t>(stream));
 }
 
+int paged_kv_copy_blocks_fp8(void* k_cache, void* v_cache, float* k_scale, float* v_scale,
+                             pkv_cache_desc cache, const int32_t* block_pairs, int32_t num_pairs,
+                             int32_t* dbg_err, void* stream) {
+  g_last_error[0] = 0;
+  const char* fn = "paged_kv_copy_blocks_fp8";
+  if (int st = check_cache(cache, fn)) return st;
+  if (cache.dtype != PKV_FP8_E4M3)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: E4M3 pools only (others take paged_kv_copy_blocks)", fn);
+  const int64_t scale_bytes = (int64_t)cache.num_kv_heads * cache.block_size * 4;
+  if (scale_bytes % 16)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: num_kv_heads * block_size must be a multiple of 4", fn);
+  if (num_pairs < 0) return fail(PKV_ERR_INVALID_ARG, "%s: num_pairs < 0", fn);
+  if (num_pairs == 0) return PKV_OK;
+  if (!k_cache || !v_cache || !k_scale || !v_scale || !block_pairs)
+    return fail(PKV_ERR_INVALID_ARG, "%s: null pointer", fn);
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_scale) || !aligned16(v_scale))
+    return fail(PKV_ERR_INVALID_ARG, "%s: pools and scales must be 16-byte aligned", fn);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (int st = launch_copy_blocks(k_cache, v_cache, cache, block_pairs, num_pairs, dbg_err, s))
+    return st;
+  return launch_copy_spans(k_scale, v_scale, scale_bytes, cache.num_blocks, block_pairs,
+                           num_pairs, dbg_err, s);
+}
+
 size_t paged_attention_decode_workspace_size(int32_t batch, int32_t num_q_heads,
                                              pkv_cache_desc cache) {
   if (check_cache(cache, "paged_attention_decode_workspace_size") != PKV_OK) return 0;

@@ -217,18 +217,25 @@ int launch_gather(const void* k_cache, const void* v_cache, const pkv_cache_desc
   return check_launch("paged_kv_gather");
 }
 
-int launch_copy_blocks(void* k_cache, void* v_cache, const pkv_cache_desc& c,
-                       const int32_t* pairs, int32_t num_pairs, int32_t* dbg, cudaStream_t s,
-                       bool skip_unset) {
-  const int es = dtype_size(c.dtype);
-  const int64_t vec_per_block = (int64_t)c.num_kv_heads * c.block_size * c.head_dim * es / 16;
+int launch_copy_spans(void* a, void* b, int64_t bytes_per_block, int32_t num_blocks,
+                      const int32_t* pairs, int32_t num_pairs, int32_t* dbg, cudaStream_t s,
+                      bool skip_unset) {
+  const int64_t vec_per_block = bytes_per_block / 16;
   const int64_t num_vec = (int64_t)num_pairs * vec_per_block;
   if (num_vec == 0) return PKV_OK;
   const int threads = 256;
   kv_copy_blocks_kernel<<<grid_for(num_vec, threads), threads, 0, s>>>(
-      static_cast<int4*>(k_cache), static_cast<int4*>(v_cache), pairs, num_vec, vec_per_block,
-      c.num_blocks, skip_unset, dbg);
+      static_cast<int4*>(a), static_cast<int4*>(b), pairs, num_vec, vec_per_block, num_blocks,
+      skip_unset, dbg);
   return check_launch("paged_kv_copy_blocks");
+}
+
+int launch_copy_blocks(void* k_cache, void* v_cache, const pkv_cache_desc& c,
+                       const int32_t* pairs, int32_t num_pairs, int32_t* dbg, cudaStream_t s,
+                       bool skip_unset) {
+  const int64_t bytes = (int64_t)c.num_kv_heads * c.block_size * c.head_dim * dtype_size(c.dtype);
+  return launch_copy_spans(k_cache, v_cache, bytes, c.num_blocks, pairs, num_pairs, dbg, s,
+                           skip_unset);
 }
 
 }  // namespace pkv

@@ -47,6 +47,11 @@ int launch_gather(const void* k_cache, const void* v_cache, const pkv_cache_desc
                   int32_t out_max_len, void* k_out, void* v_out, int32_t* dbg, cudaStream_t s);
 
 // With skip_unset, pairs (-1, -1) copy nothing (a list with holes).
+// Copies num_pairs (src, dst) spans of bytes_per_block (a multiple of 16)
+// bytes in two arrays of num_blocks spans each (pools, or their row scales).
+int launch_copy_spans(void* a, void* b, int64_t bytes_per_block, int32_t num_blocks,
+                      const int32_t* pairs, int32_t num_pairs, int32_t* dbg, cudaStream_t s,
+                      bool skip_unset = false);
 int launch_copy_blocks(void* k_cache, void* v_cache, const pkv_cache_desc& c,
                        const int32_t* pairs, int32_t num_pairs, int32_t* dbg, cudaStream_t s,
                        bool skip_unset = false);

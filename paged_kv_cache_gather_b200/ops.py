@@ -239,6 +239,24 @@ def paged_kv_copy_blocks(k_cache, v_cache, block_pairs, dbg_err=None):
                                          _stream()))
 
 
+def paged_kv_copy_blocks_fp8(k_cache, v_cache, k_scale, v_scale, block_pairs, dbg_err=None):
+    """Copy-on-write on E4M3 pools: the codes and the row scales of block src
+    go to block dst for each (src, dst) row of ``block_pairs``."""
+    _check_pool(k_cache, v_cache)
+    _check(k_cache.dtype in (torch.uint8, torch.float8_e4m3fn), "pools must hold E4M3 codes")
+    _check_scales(k_scale, v_scale, k_cache)
+    dev = k_cache.device
+    if isinstance(block_pairs, (list, tuple)):
+        block_pairs = torch.tensor(block_pairs, dtype=torch.int32, device=dev).view(-1, 2)
+    _check(block_pairs.dtype == torch.int32 and block_pairs.device == dev and
+           block_pairs.is_contiguous() and block_pairs.dim() == 2 and block_pairs.shape[1] == 2,
+           "block_pairs must be a contiguous int32 [n, 2] tensor on the device")
+    L.check(L.lib().paged_kv_copy_blocks_fp8(_ptr(k_cache), _ptr(v_cache), _ptr(k_scale),
+                                             _ptr(v_scale), cache_desc(k_cache),
+                                             _ptr(block_pairs), block_pairs.shape[0],
+                                             _ptr(dbg_err), _stream()))
+
+
 def decode_workspace_size(batch, num_q_heads, k_cache):
     return int(L.lib().paged_attention_decode_workspace_size(batch, num_q_heads,
                                                              cache_desc(k_cache)))
@@ -388,12 +406,17 @@ class DevicePool:
 
 
 def paged_kv_reserve_slots(k_cache, v_cache, block_tables, seq_lens, num_new, pool: DevicePool,
-                           num_tokens, dbg_err=None):
+                           num_tokens, dbg_err=None, k_scale=None, v_scale=None):
     """Reserve slots for ``num_new[b]`` new tokens of every sequence on the
     device (new blocks from the pool, copy-on-write of shared partly filled
     blocks). Updates block_tables, seq_lens and the pool in place. Returns
-    (slot_mapping int64 [num_tokens], cow_pairs int32 [B, 2])."""
+    (slot_mapping int64 [num_tokens], cow_pairs int32 [B, 2]). E4M3 pools pass
+    their row scales, which are copied with the codes."""
     _check_pool(k_cache, v_cache)
+    fp8 = k_cache.dtype in (torch.uint8, torch.float8_e4m3fn)
+    if fp8 or k_scale is not None or v_scale is not None:
+        _check(fp8, "row scales belong to E4M3 pools")
+        _check_scales(k_scale, v_scale, k_cache)
     dev = k_cache.device
     for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens"), (num_new, "num_new"),
                     (pool.free_stack, "free_stack"), (pool.free_top, "free_top"),
@@ -407,11 +430,15 @@ def paged_kv_reserve_slots(k_cache, v_cache, block_tables, seq_lens, num_new, po
            pool.scratch.numel() >= 2 * nb, "pool arrays are smaller than the pool")
     slots = torch.empty(max(int(num_tokens), 1), dtype=torch.int64, device=dev)
     pairs = torch.empty(B, 2, dtype=torch.int32, device=dev)
-    L.check(L.lib().paged_kv_reserve_slots(
-        _ptr(k_cache), _ptr(v_cache), cache_desc(k_cache), _ptr(block_tables),
-        block_tables.shape[1], _ptr(seq_lens), _ptr(num_new), B, _ptr(pool.free_stack),
-        _ptr(pool.free_top), _ptr(pool.refcount), _ptr(pool.scratch), _ptr(slots),
-        int(num_tokens), _ptr(pairs), _ptr(dbg_err), _stream()))
+    tail = (cache_desc(k_cache), _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens),
+            _ptr(num_new), B, _ptr(pool.free_stack), _ptr(pool.free_top), _ptr(pool.refcount),
+            _ptr(pool.scratch), _ptr(slots), int(num_tokens), _ptr(pairs), _ptr(dbg_err),
+            _stream())
+    if fp8:
+        L.check(L.lib().paged_kv_reserve_slots_fp8(_ptr(k_cache), _ptr(v_cache), _ptr(k_scale),
+                                                   _ptr(v_scale), *tail))
+    else:
+        L.check(L.lib().paged_kv_reserve_slots(_ptr(k_cache), _ptr(v_cache), *tail))
     return slots[:int(num_tokens)], pairs
 
 

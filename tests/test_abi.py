@@ -223,3 +223,25 @@ def test_debug_entries_reject_bad_arguments(lib):
     assert lib.pkv_debug_exp2(FAKE, FAKE, -1, None) == L.PKV_ERR_INVALID_ARG
     assert lib.pkv_debug_exp2(FAKE, FAKE, 0, None) == L.PKV_OK
     assert lib.pkv_debug_wait_timeout(None, None, None) == L.PKV_ERR_INVALID_ARG
+
+
+def test_fp8_copy_and_reserve_argument_checks(lib):
+    fp8 = desc(dt=E4M3)
+
+    def cp(c=fp8, ks=FAKE, n=2, pairs=FAKE):
+        return lib.paged_kv_copy_blocks_fp8(FAKE, FAKE, ks, FAKE, c, pairs, n, None, None)
+    assert cp(c=desc()) == L.PKV_ERR_UNSUPPORTED                    # bf16 pools: plain copy
+    assert cp(c=desc(dt=E4M3, bs=2, h=1)) == L.PKV_ERR_UNSUPPORTED  # scale spans of 8 bytes
+    assert cp(n=-1) == L.PKV_ERR_INVALID_ARG
+    assert cp(ks=None) == L.PKV_ERR_INVALID_ARG
+    assert cp(pairs=None) == L.PKV_ERR_INVALID_ARG
+    assert cp(ks=ctypes.c_void_p(0x10004)) == L.PKV_ERR_INVALID_ARG
+    assert cp(n=0) == L.PKV_OK
+
+    def rs(c=fp8, ks=FAKE, B=4):
+        return lib.paged_kv_reserve_slots_fp8(FAKE, FAKE, ks, FAKE, c, FAKE, 8, FAKE, FAKE, B,
+                                              FAKE, FAKE, FAKE, FAKE, FAKE, 4, FAKE, None, None)
+    assert rs(c=desc()) == L.PKV_ERR_UNSUPPORTED
+    assert rs(ks=None) == L.PKV_ERR_INVALID_ARG
+    assert rs(B=8193) == L.PKV_ERR_UNSUPPORTED
+    assert rs(B=0) == L.PKV_OK
