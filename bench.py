@@ -177,6 +177,34 @@ def decode_plan(case, steps):
     return torch.from_numpy(tab), torch.from_numpy(lens), torch.from_numpy(slots)
 
 
+def causal_pairs(ctx_lens, q_lens):
+    """(query, key) pairs a causal chunked prefill computes: chunk row i of a
+    sequence with C cached tokens sees C + i + 1 keys."""
+    C = np.asarray(ctx_lens, dtype=np.int64)
+    Q = np.asarray(q_lens, dtype=np.int64)
+    return int((Q * C + Q * (Q + 1) // 2).sum())
+
+
+def document_pairs(ctx_lens, q_lens, doc_offsets, doc_starts):
+    """Pairs a chunked prefill computes under the document mask: chunk row at
+    position p sees the keys from the start of its document to p (every
+    sequence's first document starts at 0)."""
+    pairs = 0
+    for b, (c, q) in enumerate(zip(ctx_lens, q_lens)):
+        starts = np.sort(np.asarray(doc_starts)[doc_offsets[b]:doc_offsets[b + 1]])
+        qpos = int(c) + np.arange(int(q))
+        ds = starts[np.searchsorted(starts, qpos, side="right") - 1]
+        pairs += int((qpos - ds + 1).sum())
+    return pairs
+
+
+def prefix_lm_pairs(ctx_lens, q_lens, prefix_len):
+    """Pairs under the prefix-LM mask (prefix_len <= C + Q): chunk row at
+    position p sees max(p + 1, prefix_len) keys."""
+    return int(sum(np.maximum(int(c) + np.arange(int(q)) + 1, int(pl)).sum()
+                   for c, q, pl in zip(ctx_lens, q_lens, prefix_len)))
+
+
 def visible_tokens(lens, wps):
     lens = np.asarray(lens, dtype=np.int64)
     w = np.asarray(wps, dtype=np.int64)
@@ -322,8 +350,7 @@ class PrefillWork:
         self.lse_e = [r[lo:rb].view(torch.float32).view(self.lse.shape) for r in self.res_d]
         C = c.ctx_lens.numpy().astype(np.int64)
         Q = c.q_lens.numpy().astype(np.int64)
-        pairs = (Q * C + Q * (Q + 1) // 2).sum()  # causally visible (query, key) pairs
-        self.flops = float(4 * c.head_dim * pairs * c.num_q_heads)
+        self.flops = float(4 * c.head_dim * causal_pairs(C, Q) * c.num_q_heads)
         self.h2d = off   # bytes actually copied per step (with alignment pads)
         self.d2h = rb
 
@@ -562,12 +589,7 @@ def mask_modifiers(dev, d=None):
     C = c.ctx_lens.numpy().astype(np.int64)
     Q = c.q_lens.numpy().astype(np.int64)
     off, st = I.document_starts((C + Q).tolist(), 77, mean_doc=4096)
-    pairs = 0
-    for b in range(len(C)):
-        starts = np.sort(st.numpy()[off[b]:off[b + 1]])
-        qpos = C[b] + np.arange(Q[b])
-        ds = starts[np.searchsorted(starts, qpos, side="right") - 1]
-        pairs += int((qpos - ds + 1).sum())
+    pairs = document_pairs(C, Q, off.numpy(), st.numpy())
     pw.mask = pkv.document(off.to(dev), st.to(dev))
     pw.prefill()
     ms = time_calls(pw.prefill, 5)
@@ -576,7 +598,7 @@ def mask_modifiers(dev, d=None):
                                 "visible_pairs_per_head": pairs,
                                 "documents": int(off[-1].item())}
     plen = C + Q // 2
-    pairs = int(sum((np.maximum(C[b] + np.arange(Q[b]) + 1, plen[b])).sum() for b in range(len(C))))
+    pairs = prefix_lm_pairs(C, Q, plen)
     pw.mask = pkv.prefix_lm(torch.from_numpy(plen.astype(np.int32)).to(dev))
     pw.prefill()
     ms = time_calls(pw.prefill, 5)
