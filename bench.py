@@ -55,7 +55,7 @@ def peaks():
 # ------------------------------------------------------------------ profiled traffic
 
 # DRAM bytes (read + write) per unit of work, from one ncu capture of each
-# kernel on a smaller case of the same workload (profiles/*.md); a full launch
+# kernel on a smaller case of the same workload (the committed ncu summaries); a full launch
 # scales it by its units. Valid only for the kernel code it was taken on: after
 # any change to that code (comments aside) the bench reports null until the
 # kernels are profiled again.

@@ -432,8 +432,10 @@ PKV_API int paged_attention_block_mask(const int32_t* ctx_lens, const int32_t* q
  * current); make that first call before any stream capture begins. Every
  * call shares the array: calls that overlap on the GPU race and give wrong
  * results, so order them on one stream. Nothing in the array needs to start
- * at zero. A problem that needs more scratch than the array holds returns
- * PKV_ERR_WORKSPACE_TOO_SMALL and launches nothing. The call allocates and
+ * at zero. A problem that needs more scratch than the array holds (more than
+ * paged_attention_decode_workspace_size reports for the same sizes) returns
+ * PKV_ERR_WORKSPACE_TOO_SMALL and launches nothing; batch < 0 returns
+ * PKV_ERR_INVALID_ARG, as the regular call does. The call allocates and
  * frees nothing.
  */
 #define PKV_NOALLOC_SCRATCH_BYTES (8u << 20)
@@ -443,15 +445,6 @@ PKV_API int paged_attention_decode_noalloc(const void* q, const void* k_cache, c
                                            int32_t batch, int32_t num_q_heads, float scale,
                                            pkv_mask_mod mask, void* out, float* lse,
                                            int32_t* dbg_err, void* stream);
-
-/*
- * pkv_debug_exp2 — diagnostic, not part of the attention API: y[i] = 2^x[i]
- * computed by the library's FMA-pipe exponential (exact base-2 range reduction
- * plus a fitted cubic; relative error <= 1e-4 for -126 <= x <= 127, exactly 0
- * below -126), a building block for taking exponentials off the MUFU unit that
- * the attention kernels do not use at present. x, y: device float32 [n].
- */
-PKV_API int pkv_debug_exp2(const float* x, float* y, int32_t n, void* stream);
 
 /*
  * pkv_debug_wait_timeout — diagnostic, not part of the attention API: one warp

@@ -27,7 +27,13 @@ physical blocks, closed forms (identical keys, a dominant key, W >= L), a
 pure-Python brute force on tiny inputs, split-and-merge of the softmax, and
 shared-vs-copied prefixes; ``tests/test_golden.py`` checks decode, prefill,
 append and gather against a worked example with hand-derived exact answers
-(``tests/golden/``). No function here is parity-unpinned.
+(``tests/golden/``). The E4M3 pools of ``oracle.fp8`` are pinned by
+``tests/test_oracle_fp8.py`` (rounding and decoding against torch's
+float8_e4m3fn, a separate implementation of the format) and
+``tests/test_oracle_fp8_placement.py`` (a hand-derived worked example in
+``tests/golden/``, a scalar brute force of the placement and the read-back,
+and planted mistakes that those checks reject). No function here is
+parity-unpinned.
 """
 
 from .attention64 import (  # noqa: F401
@@ -43,6 +49,7 @@ from .attention64 import (  # noqa: F401
     paged_decode,
     paged_prefill,
     paged_prefill_rows,
+    paged_prefill_tile,
     paged_decode_rows,
     kv_append,
     kv_gather,

@@ -252,6 +252,51 @@ def paged_prefill_rows(q, k_new, v_new, k_cache, v_cache, block_tables, ctx_lens
     return res
 
 
+def paged_prefill_tile(q, k_new, v_new, k_cache, v_cache, block_tables, ctx_lens, q_lens,
+                      scale, kind, b, i0, i1, heads=None, window=0, window_per_seq=None,
+                      window_per_head=None, prefix_len=None, doc_offsets=None,
+                      doc_starts=None):
+    """Chunked prefill of new queries i0 .. i1-1 of sequence b, for the given
+    query heads (all when None): out [i1-i0, len(heads), d], lse [i1-i0,
+    len(heads)] (float64). The same definition as ``paged_prefill``, evaluated
+    on one block of query rows at a time (a whole query tile of a long
+    sequence costs one matrix product per head)."""
+    q = _f64(q)
+    ctx = _i64(ctx_lens)
+    ql = _i64(q_lens)
+    tables = _i64(block_tables)
+    Hq = q.shape[1]
+    Hkv = k_cache.shape[1]
+    bs = k_cache.shape[2]
+    g = Hq // Hkv
+    heads = list(range(Hq)) if heads is None else list(heads)
+    starts = np.concatenate([[0], np.cumsum(ql)])
+    C, Q = int(ctx[b]), int(ql[b])
+    i1 = min(int(i1), Q)
+    s0 = int(starts[b])
+    kn = _f64(k_new[s0:s0 + Q])
+    vn = _f64(v_new[s0:s0 + Q])
+    d = q.shape[2]
+    out = np.zeros((max(i1 - i0, 0), len(heads), d))
+    lse = np.zeros((max(i1 - i0, 0), len(heads)))
+    by_kv = {}
+    for j, h in enumerate(heads):
+        kvh = h // g
+        if kvh not in by_kv:
+            kctx = resolve_block_table(k_cache[:, kvh:kvh + 1], tables[b], C, bs)[:, 0]
+            vctx = resolve_block_table(v_cache[:, kvh:kvh + 1], tables[b], C, bs)[:, 0]
+            by_kv[kvh] = (np.concatenate([kctx, kn[:, kvh]], axis=0),
+                          np.concatenate([vctx, vn[:, kvh]], axis=0))
+        K, V = by_kv[kvh]
+        w, P, dst = _mask_of(b, h, window, window_per_seq, window_per_head, prefix_len,
+                             doc_offsets, doc_starts)
+        o, l = masked_attention(q[s0 + i0:s0 + i1, h], K, V, C + np.arange(i0, i1),
+                                np.arange(C + Q), scale, kind, w, P, dst)
+        out[:, j] = o
+        lse[:, j] = l
+    return out, lse
+
+
 def paged_prefill(q, k_new, v_new, k_cache, v_cache, block_tables, ctx_lens, q_lens,
                   scale, kind, window=0, window_per_seq=None, window_per_head=None,
                   prefix_len=None, doc_offsets=None, doc_starts=None):

@@ -19,6 +19,12 @@ the subnormals ``m * 2**-9``; code 0x7F / 0xFF is NaN (there is no infinity).
 Pins (``tests/test_oracle_fp8.py``): rounding against torch's float8_e4m3fn
 cast over normals, subnormals and ties; decode against torch's reinterpretation
 of all 256 codes; encode(decode(c)) == c; the relative error bound 2**-4.
+``kv_append_fp8`` and ``dequantize_pool`` (``tests/test_oracle_fp8_placement.py``):
+a worked example with hand-derived codes, scales and read-back values
+(``tests/golden/e4m3_append_example.json``), a scalar brute force of the
+placement (block ``slot // bs``, row ``slot % bs``, every KV head) and of the
+read-back, and planted mistakes (head swapped, block and row swapped, one
+pool's scales for both, a scale per block, the scale on the wrong axis).
 """
 
 import numpy as np

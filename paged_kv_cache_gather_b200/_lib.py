@@ -40,6 +40,9 @@ PKV_BLOCK_SKIP = 0
 PKV_BLOCK_PARTIAL = 1
 PKV_BLOCK_FULL = 2
 
+# size of the fixed scratch of paged_attention_decode_noalloc (include/pagedkv.h)
+PKV_NOALLOC_SCRATCH_BYTES = 8 << 20
+
 # every symbol the header declares; the CPU test checks that all are exported
 EXPORTS = (
     "paged_kv_append",
@@ -58,7 +61,6 @@ EXPORTS = (
     "paged_kv_reserve_slots_fp8",
     "paged_kv_append_fp8",
     "paged_attention_decode_fp8",
-    "pkv_debug_exp2",
     "pkv_debug_wait_timeout",
     "pkv_status_string",
     "pkv_last_error",
@@ -141,8 +143,6 @@ def _declare(lib):
                                                _vp, _i32, _i32, _f32, MaskModC, _vp, _vp, _vp,
                                                _sz, _vp, _vp]
     lib.paged_attention_decode_fp8.restype = ctypes.c_int
-    lib.pkv_debug_exp2.argtypes = [_vp, _vp, _i32, _vp]
-    lib.pkv_debug_exp2.restype = ctypes.c_int
     lib.pkv_debug_wait_timeout.argtypes = [_vp, _vp, _vp]
     lib.pkv_debug_wait_timeout.restype = ctypes.c_int
     lib.pkv_status_string.argtypes = [ctypes.c_int]

@@ -234,7 +234,7 @@ int paged_kv_copy_blocks_fp8(void* k_cache, void* v_cache, float* k_scale, float
 size_t paged_attention_decode_workspace_size(int32_t batch, int32_t num_q_heads,
                                              pkv_cache_desc cache) {
   if (check_cache(cache, "paged_attention_decode_workspace_size") != PKV_OK) return 0;
-  if (num_q_heads <= 0 || num_q_heads % cache.num_kv_heads) return 0;
+  if (batch < 0 || num_q_heads <= 0 || num_q_heads % cache.num_kv_heads) return 0;
   return decode_workspace_size(batch, num_q_heads, cache);
 }
 
@@ -350,20 +350,6 @@ int paged_attention_prefill(const void* q, const void* k_new, const void* v_new,
                 ctx_lens, q_lens, batch, total_q, num_q_heads, scale, mask, out,
                 lse,      dbg_err, static_cast<cudaStream_t>(stream)};
   return launch_prefill(a);
-}
-
-__global__ void debug_exp2_kernel(const float* x, float* y, int n) {
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
-    y[i] = exp2_fma(x[i]);
-}
-
-int pkv_debug_exp2(const float* x, float* y, int32_t n, void* stream) {
-  g_last_error[0] = 0;
-  if (n < 0 || (n > 0 && (!x || !y))) return fail(PKV_ERR_INVALID_ARG, "pkv_debug_exp2: bad args");
-  if (n == 0) return PKV_OK;
-  debug_exp2_kernel<<<(n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184, 256, 0,
-                      static_cast<cudaStream_t>(stream)>>>(x, y, n);
-  return check_launch("pkv_debug_exp2");
 }
 
 // One warp waits on an mbarrier that nothing arrives on, through the same

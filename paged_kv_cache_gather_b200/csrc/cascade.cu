@@ -34,11 +34,9 @@
 //    merges the two, and writes bf16 out and the LSE.
 #include <climits>
 #include <cmath>
-#include <cstdlib>
 
 #include "pkv_common.cuh"
 #include "pkv_internal.h"
-#include "tc_sm100.cuh"
 
 namespace pkv {
 
@@ -73,7 +71,6 @@ struct GroupedParams {
   int32_t num_q_heads;
   int32_t bs_shift;
   int32_t num_blocks;
-  int32_t pool_rows;           // num_blocks * Hkv * block_size (first out-of-bounds row)
   float scale_log2;
   __nv_bfloat16* out;
   float* lse;
@@ -696,512 +693,6 @@ __global__ void __launch_bounds__(128) grouped_combine_kernel(const GroupedParam
   if (p.lse && lane == 0) p.lse[row] = lse;
 }
 
-// ------------------------------------------------------------------ tensor-core variant
-//
-// grouped_decode_tc_kernel: the same work list in 128-token tiles, one CTA per
-// SM. S^T = K Q^T puts the tile's 128 tokens on M (TMEM lanes) and the
-// segment's query rows on N (32 columns), O^T = V^T P^T puts head_dim on M and
-// the rows on N (64 columns, 32 of them zero). Warps 0-3 own one token (for S)
-// or one head_dim index (for O) each: the softmax reduces each column over the
-// 128 lanes (a butterfly inside each warp, then four partials in shared
-// memory), writes P^T as the shared-memory B operand, and rescales O only when
-// a column's maximum grows by more than 2^8. Warp 4 issues the TMA loads of
-// K and V (16-row boxes per paged block, two stages of 64 KB), warp 5 issues
-// the MMAs and owns tensor memory.
-namespace {
-
-constexpr int kTT = 128;                  // tokens per tile
-constexpr int kTCThreads = 192;
-constexpr int kTCHalf = kTT * 128;        // one 64-column half of a K or V tile: 16 KB
-constexpr int kTCTile = 2 * kTCHalf;      // 32 KB
-constexpr int kTCStage = 2 * kTCTile;     // K then V: 64 KB
-constexpr int kTCQHalf = kRows * 128;     // 4 KB
-constexpr int kTCPBuf = kTT * 128;        // P^T: 128 tokens x 64 bf16 columns
-constexpr int kTCPV = 64;                 // N of the P V product (rows 32..63 are zero)
-constexpr float kTCRescale = 8.f;         // log2 units
-
-struct TCLayout {
-  static constexpr int kKV = 0;
-  static constexpr int kQ = 2 * kTCStage;
-  static constexpr int kP = kQ + 2 * kTCQHalf;
-  static constexpr int kRed = kP + 2 * kTCPBuf;        // float [2][4][32]
-  static constexpr int kRed2 = kRed + 2 * 4 * 32 * 4;  // float [4][32]
-  static constexpr int kBars = kRed2 + 4 * 32 * 4;
-  static constexpr int kNumBars = 24;
-  static constexpr int kTmemSlot = kBars + kNumBars * 8;
-  static constexpr int kAbort = kTmemSlot + 8;
-  static constexpr int kBytes = kAbort + 8;
-};
-
-// K and V have separate 2-stage rings: a K stage is free once S of its tile
-// is done, so K loads (and S) run a tile ahead of P V.
-enum : int {
-  TB_Q_FULL = 0,
-  TB_Q_EMPTY = 1,
-  TB_K_FULL = 2,               // + stage
-  TB_K_EMPTY = 4,              // + stage
-  TB_V_FULL = 6,               // + stage
-  TB_V_EMPTY = 8,              // + stage
-  TB_S_FULL = 10,              // + buffer
-  TB_S_FREE = 12,              // + buffer
-  TB_P_FULL = 14,              // + buffer
-  TB_PV_DONE = 16,             // + buffer
-  TB_O_FULL = 18,
-  TB_O_FREE = 19,
-  TB_RED = 20,
-  TB_SUM = 21,
-};
-
-// Warp-collective bounded wait (every lane returns the same answer); with
-// `all_lanes` every lane polls, so each has acquired what the phase publishes.
-__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, int32_t* dbg,
-                                        int* abort_flag, bool all_lanes) {
-  bool ok = true;
-  if (all_lanes || (threadIdx.x & 31) == 0)
-    ok = *reinterpret_cast<volatile int*>(abort_flag) == 0 && mbar_wait(bar, parity);
-  ok = __all_sync(0xffffffffu, ok);
-  __syncwarp();
-  if (!ok && (threadIdx.x & 31) == 0) {
-    flag_error(dbg, PKV_DBG_TIMEOUT);
-    *reinterpret_cast<volatile int*>(abort_flag) = 1;
-  }
-  return ok;
-}
-
-__device__ __forceinline__ void mbar_arrive_tc(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-// Per-tile facts every role derives the same way.
-struct TileInfo {
-  int tok0;           // position of the tile's first token
-  bool seg_begin, seg_end;
-  bool fix;           // a 16-row box straddles the end: its rows past it are zeroed in V
-};
-
-}  // namespace
-
-__global__ void __launch_bounds__(kTCThreads, 1)
-    grouped_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
-                             const __grid_constant__ CUtensorMap vmap, const GroupedParams p) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  using L = TCLayout;
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int lane = tid & 31;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-  auto bar = [&](int i) { return smem_u32(bars + i); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
-  int* abort_flag = reinterpret_cast<int*>(smem + L::kAbort);
-
-  // this CTA's contiguous range of the flat list (every warp derives it)
-  const int64_t T =
-      (int64_t)total_tiles<kTT>(p, lane, (blockIdx.x == 0 && warp == 0) ? p.ws_prefix : nullptr) *
-      p.num_kv_heads;
-  const int W = workers_for(T, p.workers);
-  const int gw = blockIdx.x;
-  int64_t start = 0, end = 0;
-  if (gw < W && T > 0) {
-    start = (int64_t)gw * T / W;
-    end = (int64_t)(gw + 1) * T / W;
-  }
-  const int64_t ntiles = end - start;
-
-  if (warp == 4) {
-    if (lane == 0) {
-      mbar_init(bar(TB_Q_FULL), 128);
-      mbar_init(bar(TB_Q_EMPTY), 1);
-      for (int s = 0; s < 2; ++s) {
-        mbar_init(bar(TB_K_FULL + s), 1);
-        mbar_init(bar(TB_K_EMPTY + s), 1);
-        mbar_init(bar(TB_V_FULL + s), 1);
-        mbar_init(bar(TB_V_EMPTY + s), 1);
-        mbar_init(bar(TB_S_FULL + s), 1);
-        mbar_init(bar(TB_S_FREE + s), 128);
-        mbar_init(bar(TB_P_FULL + s), 128);
-        mbar_init(bar(TB_PV_DONE + s), 1);
-      }
-      mbar_init(bar(TB_O_FULL), 1);
-      mbar_init(bar(TB_O_FREE), 128);
-      mbar_init(bar(TB_RED), 128);
-      mbar_init(bar(TB_SUM), 128);
-      *abort_flag = 0;
-      fence_barrier_init();
-      prefetch_tmap(&kmap);
-      prefetch_tmap(&vmap);
-    }
-  } else if (warp == 5) {
-    tc::tmem_alloc(smem_u32(tmem_slot), 128);
-    tc::tmem_relinquish();
-  } else {
-    // columns 32..63 of both P^T buffers stay zero (rows 32..63 of the P V product)
-    for (int i = tid; i < 2 * kTT * 4; i += 128) {
-      const int buf = i / (kTT * 4), r = (i / 4) % kTT, ch = 4 + (i & 3);
-      *reinterpret_cast<int4*>(smem + L::kP + buf * kTCPBuf + r * 128 + ((ch ^ (r & 7)) << 4)) =
-          make_int4(0, 0, 0, 0);
-    }
-    fence_proxy_async_smem();
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tmem = *tmem_slot;
-
-  if (ntiles > 0) {
-    Cursor cur;
-    {
-      int i;
-      int64_t before;
-      find_item<kTT>(p, lane, start, i, before);
-      cur.i = i;
-      cur.it = item_of<kTT>(p, i);
-      const int64_t off = start - before;
-      cur.kvh = (int)(off / cur.it.n);
-      cur.seg_first = before + (int64_t)cur.kvh * cur.it.n;
-      cur.t = start;
-    }
-    const int box_rows = p.bs_shift >= 4 ? 16 : (1 << p.bs_shift);
-    auto info = [&](const Cursor& c, int64_t k) {
-      TileInfo ti;
-      ti.tok0 = (c.it.t0 + (int)(c.t - c.seg_first)) * kTT;
-      ti.seg_begin = (k == 0) || (c.t == c.seg_first);
-      ti.seg_end = (k == ntiles - 1) || (c.t + 1 == c.seg_first + c.it.n);
-      ti.fix = ti.tok0 < c.it.hi && c.it.hi < ti.tok0 + kTT && (c.it.hi % box_rows) != 0;
-      return ti;
-    };
-
-    if (warp == 4) {
-      // ============================================================ TMA producer
-      const int nbox = kTT / box_rows;
-      const int bs_mask = (1 << p.bs_shift) - 1;
-      // block id of this lane's box of a tile (-2: outside [lo, hi), zero fill)
-      auto fetch = [&](const Cursor& c) -> int {
-        if (lane >= nbox) return -2;
-        const int pos = (c.it.t0 + (int)(c.t - c.seg_first)) * kTT + lane * box_rows;
-        if (pos >= c.it.hi || pos + box_rows <= c.it.lo) return -2;
-        const int j = pos >> p.bs_shift;
-        return j < p.max_blocks ? __ldg(p.tables + (int64_t)c.it.lead * p.max_blocks + j) : -1;
-      };
-      // K of tile k is issued one step before V of tile k-1
-      auto load_boxes = [&](const Cursor& c, int id, int stage, bool is_v) {
-        if (lane >= nbox) return;
-        int row = p.pool_rows;  // out of bounds: TMA fills zeros
-        if (id >= 0 && id < p.num_blocks)
-          row = ((id * p.num_kv_heads + c.kvh) << p.bs_shift) +
-                (((c.it.t0 + (int)(c.t - c.seg_first)) * kTT + lane * box_rows) & bs_mask);
-        else if (id != -2)
-          flag_error(p.dbg, PKV_DBG_BLOCK_ID);
-        const uint32_t dst = smem_u32(smem + L::kKV + stage * kTCStage + (is_v ? kTCTile : 0)) +
-                             lane * box_rows * 128;
-        const int b = (is_v ? TB_V_FULL : TB_K_FULL) + stage;
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          tma_load_2d(dst + h * kTCHalf, is_v ? &vmap : &kmap, h * 64, row, bar(b));
-      };
-      Cursor pc = cur, pprev = cur;
-      int id_cur = fetch(pc), id_prev = -2;
-      for (int64_t k = 0; k <= ntiles; ++k) {
-        Cursor nx = pc;
-        int id_next = -2;
-        if (k < ntiles) {
-          const int s = (int)(k & 1);
-          if (k >= 2 &&
-              !tc_wait(bar(TB_K_EMPTY + s), ((k >> 1) - 1) & 1, p.dbg, abort_flag, false))
-            break;
-          if (lane == 0) mbar_arrive_expect_tx(bar(TB_K_FULL + s), kTCTile);
-          __syncwarp();
-          load_boxes(pc, id_cur, s, false);
-          cursor_advance<kTT>(p, nx);
-          id_next = (k + 1 < ntiles) ? fetch(nx) : -2;
-        }
-        if (k >= 1) {
-          const int64_t j = k - 1;
-          const int s = (int)(j & 1);
-          if (j >= 2 &&
-              !tc_wait(bar(TB_V_EMPTY + s), ((j >> 1) - 1) & 1, p.dbg, abort_flag, false))
-            break;
-          if (lane == 0) mbar_arrive_expect_tx(bar(TB_V_FULL + s), kTCTile);
-          __syncwarp();
-          load_boxes(pprev, id_prev, s, true);
-        }
-        pprev = pc;
-        id_prev = id_cur;
-        pc = nx;
-        id_cur = id_next;
-      }
-    } else if (warp == 5) {
-      // ============================================================ MMA issuer
-      const uint32_t idesc_s = tc::idesc_bf16(kTT, kRows, false, false);
-      const uint32_t idesc_o = tc::idesc_bf16(128, kTCPV, true, true);
-      const uint32_t kv0 = smem_u32(smem + L::kKV);
-      const uint64_t dq = tc::smem_desc(smem_u32(smem + L::kQ), 16, 1024, tc::kSwizzle128B);
-      const uint64_t dk0 = tc::smem_desc(kv0, 16, 1024, tc::kSwizzle128B);
-      const uint64_t dv0 = tc::smem_desc(kv0 + kTCTile, kTCHalf, 1024, tc::kSwizzle128B);
-      const uint64_t dp0 = tc::smem_desc(smem_u32(smem + L::kP), kTCHalf, 1024, tc::kSwizzle128B);
-      constexpr uint64_t kStageStep = (uint64_t)kTCStage >> 4;
-      constexpr uint64_t kPStep = (uint64_t)kTCPBuf >> 4;
-      const uint32_t O = tmem + 64;
-      int sg = 0;
-      TileInfo pti{};
-      int psg = 0;
-      bool ok = true;
-      auto do_pv = [&](int64_t j, const TileInfo& t, int jsg) -> bool {
-        const int s = (int)(j & 1);
-        if (!tc_wait(bar(TB_P_FULL + s), (j >> 1) & 1, p.dbg, abort_flag, false)) return false;
-        if (!tc_wait(bar(TB_V_FULL + s), (j >> 1) & 1, p.dbg, abort_flag, false)) return false;
-        if (t.seg_begin && jsg > 0 &&
-            !tc_wait(bar(TB_O_FREE), (jsg - 1) & 1, p.dbg, abort_flag, false))
-          return false;
-        tc::fence_after_sync();
-        if (lane == 0) {
-#pragma unroll
-          for (int kk = 0; kk < kTT / 16; ++kk)
-            tc::mma_ss(O, dv0 + (uint64_t)s * kStageStep + (uint64_t)(kk * (2048 >> 4)),
-                       dp0 + (uint64_t)s * kPStep + (uint64_t)(kk * (2048 >> 4)), idesc_o,
-                       !(t.seg_begin && kk == 0));
-          tc::commit(bar(TB_V_EMPTY + s));
-          tc::commit(bar(TB_PV_DONE + s));
-          if (t.seg_end) tc::commit(bar(TB_O_FULL));
-        }
-        __syncwarp();
-        return true;
-      };
-      for (int64_t k = 0; k < ntiles; ++k) {
-        const int s = (int)(k & 1);
-        const TileInfo t = info(cur, k);
-        // the previous piece's last P V goes first: its epilogue gates the next query tile
-        if (k >= 1 && t.seg_begin && !(ok = do_pv(k - 1, pti, psg))) break;
-        if (t.seg_begin) {
-          if (!(ok = tc_wait(bar(TB_Q_FULL), sg & 1, p.dbg, abort_flag, false))) break;
-          ++sg;
-        }
-        if (!(ok = tc_wait(bar(TB_K_FULL + s), (k >> 1) & 1, p.dbg, abort_flag, false))) break;
-        if (k >= 2 &&
-            !(ok = tc_wait(bar(TB_S_FREE + s), ((k >> 1) - 1) & 1, p.dbg, abort_flag, false)))
-          break;
-        tc::fence_after_sync();
-        if (lane == 0) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ok_ = (uint64_t)((kk >> 2) * (kTCHalf >> 4) + (kk & 3) * 2);
-            const uint64_t oq = (uint64_t)((kk >> 2) * (kTCQHalf >> 4) + (kk & 3) * 2);
-            tc::mma_ss(tmem + s * kRows, dk0 + (uint64_t)s * kStageStep + ok_, dq + oq, idesc_s,
-                       kk > 0);
-          }
-          tc::commit(bar(TB_S_FULL + s));
-          tc::commit(bar(TB_K_EMPTY + s));
-          if (t.seg_end) tc::commit(bar(TB_Q_EMPTY));
-        }
-        __syncwarp();
-        if (k >= 1 && !t.seg_begin && !(ok = do_pv(k - 1, pti, psg))) break;
-        pti = t;
-        psg = sg - 1;
-        cursor_advance<kTT>(p, cur);
-      }
-      if (ok) do_pv(ntiles - 1, pti, psg);
-    } else {
-      // ============================================================ softmax / epilogue
-      float* red = reinterpret_cast<float*>(smem + L::kRed);
-      float* red2 = reinterpret_cast<float*>(smem + L::kRed2);
-      const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-      const int64_t rows_all = (int64_t)p.batch * p.num_q_heads;
-      float m = -INFINITY;  // running maximum of column `lane` (scaled, base 2)
-      float lsum[kRows];    // this thread's share of every column's sum
-#pragma unroll
-      for (int c = 0; c < kRows; ++c) lsum[c] = 0.f;
-      int sg = 0, piece = 0;
-      int64_t piece_start = start;
-      for (int64_t k = 0; k < ntiles; ++k) {
-        const int sb = (int)(k & 1);
-        const TileInfo t = info(cur, k);
-        if (t.seg_begin) {
-          if (sg > 0 && !tc_wait(bar(TB_Q_EMPTY), (sg - 1) & 1, p.dbg, abort_flag, true)) break;
-          // the piece's query rows, K-major with 128-byte swizzle, zero past its rows
-          const int r = tid >> 2;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int c = (tid & 3) * 4 + j;
-            int4 v = make_int4(0, 0, 0, 0);
-            if (r < cur.it.rows) {
-              int b, h;
-              row_target(p, cur.it, cur.kvh, r, b, h);
-              v = __ldg(reinterpret_cast<const int4*>(p.q + ((int64_t)b * p.num_q_heads + h) * kD) +
-                        c);
-            }
-            *reinterpret_cast<int4*>(smem + L::kQ + (c >> 3) * kTCQHalf + r * 128 +
-                                     (((c & 7) ^ (r & 7)) << 4)) = v;
-          }
-          fence_proxy_async_smem();
-          mbar_arrive_tc(bar(TB_Q_FULL));
-          m = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < kRows; ++c) lsum[c] = 0.f;
-          piece_start = cur.t;
-          ++sg;
-        }
-        if (!tc_wait(bar(TB_S_FULL + sb), (k >> 1) & 1, p.dbg, abort_flag, true)) break;
-        tc::fence_after_sync();
-        float x[kRows];
-        {
-          uint32_t sr[32];
-          tc::ld32(tmem + lane_base + sb * kRows, sr);
-          tc::wait_ld();
-          tc::fence_before_sync();
-          mbar_arrive_tc(bar(TB_S_FREE + sb));
-          const int pos = t.tok0 + tid;
-          const bool live = pos >= cur.it.lo && pos < cur.it.hi;
-#pragma unroll
-          for (int c = 0; c < kRows; ++c)
-            x[c] = live ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
-        }
-        // column maxima over the warp's 32 tokens: after the butterfly lane l holds column l
-        float v[kRows];
-#pragma unroll
-        for (int c = 0; c < kRows; ++c) v[c] = x[c];
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-          const bool up = (lane & o) != 0;
-#pragma unroll
-          for (int i = 0; i < o; ++i) {
-            const float keep = up ? v[i + o] : v[i];
-            const float send = up ? v[i] : v[i + o];
-            v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
-          }
-        }
-        red[sb * 128 + warp * 32 + lane] = v[0];
-        mbar_arrive_tc(bar(TB_RED));
-        if (!tc_wait(bar(TB_RED), k & 1, p.dbg, abort_flag, true)) break;
-        const float* rr = red + sb * 128;
-        const float cm = fmaxf(fmaxf(rr[lane], rr[32 + lane]), fmaxf(rr[64 + lane], rr[96 + lane]));
-        float alpha = 1.f;
-        if (cm > m + kTCRescale || (m == -INFINITY && cm != -INFINITY)) {
-          alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - cm);
-          m = cm;
-        }
-        const bool resc = __any_sync(0xffffffffu, alpha != 1.f);
-        uint32_t pk[kRows / 2];
-#pragma unroll
-        for (int c = 0; c < kRows; c += 2) {
-          const float m0 = __shfl_sync(0xffffffffu, m, c), m1 = __shfl_sync(0xffffffffu, m, c + 1);
-          const float e0 = fast_exp2(x[c] - (m0 == -INFINITY ? 0.f : m0));
-          const float e1 = fast_exp2(x[c + 1] - (m1 == -INFINITY ? 0.f : m1));
-          if (resc) {
-            lsum[c] = lsum[c] * __shfl_sync(0xffffffffu, alpha, c) + e0;
-            lsum[c + 1] = lsum[c + 1] * __shfl_sync(0xffffffffu, alpha, c + 1) + e1;
-          } else {
-            lsum[c] += e0;
-            lsum[c + 1] += e1;
-          }
-          pk[c / 2] = pack_bf16x2(e0, e1);
-        }
-        // P^T row of this token (64 bytes), once P V of two tiles ago has read the buffer
-        if (k >= 2 &&
-            !tc_wait(bar(TB_PV_DONE + sb), ((k >> 1) - 1) & 1, p.dbg, abort_flag, true))
-          break;
-        uint8_t* prow = smem + L::kP + sb * kTCPBuf + tid * 128;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-          *reinterpret_cast<uint4*>(prow + ((ch ^ (tid & 7)) << 4)) =
-              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        if (t.fix) {
-          // pool rows past the end in the box holding it: zero them in V before P V
-          if (!tc_wait(bar(TB_V_FULL + sb), (k >> 1) & 1, p.dbg, abort_flag, true)) break;
-          const int r0 = cur.it.hi - t.tok0;
-          const int r1 = min(kTT, (r0 / box_rows + 1) * box_rows);
-          uint8_t* vb = smem + L::kKV + sb * kTCStage + kTCTile;
-          for (int i = tid; i < (r1 - r0) * 16; i += 128) {
-            const int rr = r0 + i / 16, h = (i / 8) & 1, ch = i & 7;
-            *reinterpret_cast<int4*>(vb + h * kTCHalf + rr * 128 + ch * 16) = make_int4(0, 0, 0, 0);
-          }
-        }
-        fence_proxy_async_smem();
-        if (resc && !t.seg_begin) {
-          // O holds earlier tiles: rescale its columns once the last P V is done
-          if (!tc_wait(bar(TB_PV_DONE + ((k - 1) & 1)), ((k - 1) >> 1) & 1, p.dbg, abort_flag,
-                       true))
-            break;
-          tc::fence_after_sync();
-          uint32_t o[32];
-          tc::ld32(tmem + lane_base + 64, o);
-          tc::wait_ld();
-#pragma unroll
-          for (int c = 0; c < kRows; ++c)
-            o[c] = __float_as_uint(__uint_as_float(o[c]) * __shfl_sync(0xffffffffu, alpha, c));
-          tc::st32(tmem + lane_base + 64, o);
-          tc::wait_st();
-        }
-        tc::fence_before_sync();
-        mbar_arrive_tc(bar(TB_P_FULL + sb));
-        if (t.seg_end) {
-          // ---- epilogue of the piece: column sums, outputs (thread = head_dim index)
-          if (!tc_wait(bar(TB_O_FULL), (sg - 1) & 1, p.dbg, abort_flag, true)) break;
-          tc::fence_after_sync();
-#pragma unroll
-          for (int c = 0; c < kRows; ++c) v[c] = lsum[c];
-#pragma unroll
-          for (int o = 16; o >= 1; o >>= 1) {
-            const bool up = (lane & o) != 0;
-#pragma unroll
-            for (int i = 0; i < o; ++i) {
-              const float keep = up ? v[i + o] : v[i];
-              const float send = up ? v[i] : v[i + o];
-              v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-            }
-          }
-          red2[warp * 32 + lane] = v[0];
-          mbar_arrive_tc(bar(TB_SUM));
-          if (!tc_wait(bar(TB_SUM), (sg - 1) & 1, p.dbg, abort_flag, true)) break;
-          const float tot = (red2[lane] + red2[32 + lane]) + (red2[64 + lane] + red2[96 + lane]);
-          const float inv = tot > 0.f ? 1.f / tot : 0.f;
-          const float lse = tot > 0.f ? m * kLn2 + logf(tot) : -INFINITY;
-          uint32_t o[32];
-          tc::ld32(tmem + lane_base + 64, o);
-          tc::wait_ld();
-          const bool whole = (piece_start == cur.seg_first) && (cur.t + 1 == cur.seg_first + cur.it.n);
-          const int kind = cur.it.prefix ? 0 : 1;
-          const int64_t slot = (int64_t)gw * 2 + piece;
-#pragma unroll
-          for (int c = 0; c < kRows; ++c) {
-            const float val = __uint_as_float(o[c]) * __shfl_sync(0xffffffffu, inv, c);
-            if (c < cur.it.rows) {
-              float* dst;
-              if (whole) {
-                int b, h;
-                row_target(p, cur.it, cur.kvh, c, b, h);
-                dst = p.whole_o + (kind * rows_all + (int64_t)b * p.num_q_heads + h) * kD;
-              } else {
-                dst = p.ws_o + (slot * kRows + c) * kD;
-              }
-              dst[tid] = val;
-            }
-          }
-          if (warp == 0 && lane < cur.it.rows) {
-            if (whole) {
-              int b, h;
-              row_target(p, cur.it, cur.kvh, lane, b, h);
-              p.whole_lse[kind * rows_all + (int64_t)b * p.num_q_heads + h] = lse;
-            } else {
-              p.ws_lse[slot * kRows + lane] = lse;
-            }
-          }
-          tc::fence_before_sync();
-          mbar_arrive_tc(bar(TB_O_FREE));
-          piece = 1;
-        }
-        cursor_advance<kTT>(p, cur);
-      }
-    }
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  if (warp == 5) {
-    tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 128);
-  }
-}
-
 namespace {
 
 // Workspace: pieces (2 per worker), whole-segment results (prefix and own
@@ -1210,19 +701,6 @@ namespace {
 struct Layout {
   size_t ws_o, ws_lse, whole_o, whole_lse, prefix, total;
 };
-
-// The mma.sync kernel is the default: on the beams workload it measured 111 us
-// per call against 177 us for the tensor-core kernel, whose CTAs drain their
-// pipeline at every segment piece (query staging, epilogue through tensor
-// memory) and most pieces here are two tiles long. PKV_GROUPED_TC=1 selects
-// the tensor-core kernel.
-bool use_tc_kernel() {
-  static int v = [] {
-    const char* e = getenv("PKV_GROUPED_TC");
-    return (e && e[0] == '1') ? 1 : 0;
-  }();
-  return v != 0;
-}
 
 Layout layout(int32_t batch, int32_t num_q_heads) {
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
@@ -1347,24 +825,8 @@ PKV_API int paged_attention_decode_shared_prefix(
   p.workers = sms * kWarps;
   p.dbg = dbg_err;
 
-  p.pool_rows = (int32_t)pool_rows;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (use_tc_kernel()) {
-    // tensor-core variant: one CTA (192 threads) per SM, 128-token tiles
-    p.workers = sms;
-    const size_t smem_tc = (size_t)TCLayout::kBytes + 1024;
-    static bool tc_attr[64] = {false};
-    if (dev >= 0 && dev < 64 && !tc_attr[dev]) {
-      if (cudaFuncSetAttribute(grouped_decode_tc_kernel,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem_tc) != cudaSuccess)
-        return check_launch("paged_attention_decode_shared_prefix: smem attribute");
-      tc_attr[dev] = true;
-    }
-    grouped_decode_tc_kernel<<<sms, kTCThreads, smem_tc, s>>>(kmap, vmap, p);
-  } else {
-    grouped_decode_kernel<<<sms, kWarps * 32, smem, s>>>(kmap, vmap, p);
-  }
+  grouped_decode_kernel<<<sms, kWarps * 32, smem, s>>>(kmap, vmap, p);
   if (int st = check_launch(fn)) return st;
   const int64_t rows = (int64_t)batch * num_q_heads;
   cudaLaunchConfig_t cfg = {};

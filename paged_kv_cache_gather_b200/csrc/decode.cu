@@ -29,7 +29,6 @@
 //    movmatrix, without a trip through shared memory.
 //  * fp32 pools use a plain CUDA-core kernel (one CTA per (b, q head)).
 #include <cmath>
-#include <cstdlib>
 
 #include "pkv_common.cuh"
 #include "pkv_internal.h"
@@ -38,7 +37,6 @@ namespace pkv {
 
 constexpr int kTile = 16;            // tokens per tile
 constexpr int kMinTilesPerWorker = 2;
-constexpr int kWarpsPerCta = 12;     // default workers (warps) per CTA, one CTA per SM
 constexpr int kMaxWarpsPerCta = 12;  // largest built bf16 variant (sizes the workspace)
 
 struct DecodeParams {
@@ -623,6 +621,9 @@ __global__ void __launch_bounds__(WPC * 32, 1)
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
   constexpr int V = D / 32;  // floats per lane
+  // launched as a programmatic dependent of the main kernel: wait until its
+  // grid has completed and its partials, prefix and outputs are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
   const int H = p.num_kv_heads;
@@ -890,51 +891,22 @@ int launch_bf16_impl(const DecodeArgs& a) {
   return check_launch("paged_attention_decode: combine");
 }
 
-// Warps per CTA (one CTA per SM) and ring depth per warp. PKV_DECODE_WARPS
-// picks another built variant (for tuning sweeps); the default is the
-// fastest measured on B200.
-int decode_warps_per_cta() {
-  static int w = [] {
-    const char* e = getenv("PKV_DECODE_WARPS");
-    int v = e ? atoi(e) : kWarpsPerCta;
-    if (v != 4 && v != 6 && v != 8 && v != 12) v = kWarpsPerCta;
-    return v;
-  }();
-  return w;
-}
-
-// Warps per CTA of the E4M3 decode (PKV_DECODE_FP8_WARPS picks another built
-// variant, for tuning sweeps).
-int decode_fp8_warps() {
-  static int w = [] {
-    const char* e = getenv("PKV_DECODE_FP8_WARPS");
-    int v = e ? atoi(e) : 16;
-    return v == 12 ? 12 : 16;  // 16 warps measured 9% faster on the ragged batch
-  }();
-  return w;
-}
-
+// Warps per CTA (one CTA per SM) and ring depth per warp, the fastest
+// measured on B200: 12 warps with 2-stage rings for bf16 head_dim 128 (192 KB
+// of ring per CTA; 4, 6 and 8 warps with deeper rings were slower), 16 warps
+// with 2-stage rings for E4M3 pools (9% faster than 12 with 3).
 template <int D>
 int launch_bf16(const DecodeArgs& a) {
-  // 192 KB of ring per CTA for head_dim 128 (8 KB stages), 160-192 KB for 64
+  const bool per_head = a.mask.kind == PKV_MASK_SLIDING && a.mask.window_per_head;
   if constexpr (D == 128) {
-    // E4M3 pools: 16 warps with 2-stage rings of 4 KB tiles (or 12 with 3) and
-    // a 4 KB work tile each, 197-201 KB per CTA
+    // E4M3 pools: 4 KB tiles and a 4 KB work tile per warp, 197-201 KB per CTA
     if (a.cache.dtype == PKV_FP8_E4M3) {
-      if (a.mask.kind == PKV_MASK_SLIDING && a.mask.window_per_head)
-        return launch_bf16_impl<D, 3, 12, true, true>(a);
-      if (decode_fp8_warps() == 16) return launch_bf16_impl<D, 2, 16, false, true>(a);
-      return launch_bf16_impl<D, 3, 12, false, true>(a);
+      if (per_head) return launch_bf16_impl<D, 3, 12, true, true>(a);
+      return launch_bf16_impl<D, 2, 16, false, true>(a);
     }
   }
-  if (a.mask.kind == PKV_MASK_SLIDING && a.mask.window_per_head)
-    return launch_bf16_impl<D, (D == 128 ? 2 : 4), 12, true>(a);
-  switch (decode_warps_per_cta()) {
-    case 6: return launch_bf16_impl<D, (D == 128 ? 4 : 8), 6, false>(a);
-    case 8: return launch_bf16_impl<D, (D == 128 ? 3 : 6), 8, false>(a);
-    case 4: return launch_bf16_impl<D, (D == 128 ? 6 : 10), 4, false>(a);
-    default: return launch_bf16_impl<D, (D == 128 ? 2 : 4), 12, false>(a);
-  }
+  if (per_head) return launch_bf16_impl<D, (D == 128 ? 2 : 4), 12, true>(a);
+  return launch_bf16_impl<D, (D == 128 ? 2 : 4), 12, false>(a);
 }
 
 }  // namespace

@@ -75,6 +75,10 @@ extern "C" PKV_API int paged_attention_decode_noalloc(
     int32_t batch, int32_t num_q_heads, float scale, pkv_mask_mod mask, void* out, float* lse,
     int32_t* dbg_err, void* stream) {
   using namespace pkv;
+  if (batch < 0) {
+    clear_last_error();
+    return fail(PKV_ERR_INVALID_ARG, "paged_attention_decode_noalloc: bad batch");
+  }
   const size_t need = paged_attention_decode_workspace_size(batch, num_q_heads, cache);
   if (need > kNoAllocScratchBytes)
     return fail(PKV_ERR_WORKSPACE_TOO_SMALL,

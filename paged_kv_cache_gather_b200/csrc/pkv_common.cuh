@@ -214,27 +214,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x on the FMA pipe, for x <= 127: a building block for moving part of a
-// softmax's exponentials off the MUFU unit (the prefill kernel measured slower
-// with it on 1/16 to 1/4 of its elements, so it does not use it). Exact base-2 range
-// reduction x = j + f, j = round(x) (via the 1.5*2^23 rounding constant),
-// f in [-1/2, 1/2]; 2^f by a cubic fitted for minimum relative error
-// (paged_kv_cache_gather_b200/fit_exp2.py: max relative error 7.5e-5, 1.0e-4
-// along this float32 path); j is added to the exponent field. x < -126
-// (including -inf) gives exactly 0.
-__device__ __forceinline__ float exp2_fma(float x) {
-  const float magic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
-  const float xc = fmaxf(x, -126.0f);
-  const float t = xc + magic;
-  const float j = t - magic;
-  const float f = xc - j;
-  float p = fmaf(5.517132208e-02f, f, 2.426105440e-01f);
-  p = fmaf(p, f, 6.932609677e-01f);
-  p = fmaf(p, f, 9.999281168e-01f);
-  const int bits = __float_as_int(p) + (__float_as_int(t) << 23);
-  return x < -126.0f ? 0.0f : __int_as_float(bits);
-}
-
 __device__ __forceinline__ void flag_error(int32_t* dbg, int32_t bit) {
   if (dbg) atomicOr(dbg, bit);
 }

@@ -220,9 +220,40 @@ def test_block_mask_and_reserve_argument_checks(lib):
 
 
 def test_debug_entries_reject_bad_arguments(lib):
-    assert lib.pkv_debug_exp2(FAKE, FAKE, -1, None) == L.PKV_ERR_INVALID_ARG
-    assert lib.pkv_debug_exp2(FAKE, FAKE, 0, None) == L.PKV_OK
     assert lib.pkv_debug_wait_timeout(None, None, None) == L.PKV_ERR_INVALID_ARG
+
+
+def noalloc(lib, B, c=None, Hq=32, q=None):
+    return lib.paged_attention_decode_noalloc(q, FAKE, FAKE, c or desc(h=8), FAKE, 4, FAKE, B, Hq,
+                                              0.1, mask(), FAKE, FAKE, None, None)
+
+
+def test_noalloc_scratch_boundary(lib):
+    """The no-allocation decode accepts exactly the problems whose scratch
+    need (the regular call's workspace size) fits its fixed array: at the
+    largest such batch the size check passes (the call then fails later, on
+    the null query, never with WORKSPACE_TOO_SMALL); one sequence more is
+    rejected by the size check. Sizes are computed for a 148-SM B200, the
+    library's count when no device is visible."""
+    c = desc(h=8)  # 32 query heads / 8 KV heads, head_dim 128: group 4
+    size = lambda b: lib.paged_attention_decode_workspace_size(b, 32, c)
+    cap = L.PKV_NOALLOC_SCRATCH_BYTES
+    lo, hi = 0, 1 << 24  # size(lo) <= cap < size(hi)
+    assert size(lo) <= cap < size(hi)
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        lo, hi = (mid, hi) if size(mid) <= cap else (lo, mid)
+    assert size(lo) <= cap < size(lo + 1)
+    assert lo > 100_000  # the fixed part (per-worker partials) leaves room for a big batch
+    assert noalloc(lib, lo) not in (L.PKV_OK, L.PKV_ERR_WORKSPACE_TOO_SMALL)
+    assert noalloc(lib, lo + 1) == L.PKV_ERR_WORKSPACE_TOO_SMALL
+    assert b"built-in scratch" in lib.pkv_last_error()
+
+
+def test_noalloc_rejects_a_negative_batch_like_the_regular_call(lib):
+    assert noalloc(lib, -5) == L.PKV_ERR_INVALID_ARG
+    assert decode(lib, B=-5)[0] == L.PKV_ERR_INVALID_ARG
+    assert lib.paged_attention_decode_workspace_size(-5, 32, desc(h=8)) == 0
 
 
 def test_fp8_copy_and_reserve_argument_checks(lib):

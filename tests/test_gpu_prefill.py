@@ -4,8 +4,9 @@ Small cases are compared in full: contexts that are empty, shorter than a
 tile, not multiples of the block or tile size; chunks of 1 token up to several
 tiles; causal, no mask and sliding windows; group sizes with two heads per CTA
 (even) and one (odd); block sizes 8..64. The long-context workload (4 x 30720
-cached + 2048 new, 32/8 heads) is checked on sampled rows the oracle computes
-one by one, plain and "peaky". Also: pool rows past the context end that hold
+cached + 2048 new, 32/8 heads) is checked on whole 128-row tiles at all 32
+heads (first, middle and last tile of every sequence) and on sampled rows
+the oracle computes one by one, plain and "peaky". Also: pool rows past the context end that hold
 NaN must not leak into the result, and bad block ids are flagged.
 """
 
@@ -158,6 +159,31 @@ def test_long_context_workload_sampled_rows(cuda_device, peaky):
     assert_attention_close(go, gl, ro, rl, torch.bfloat16, case.name)
     # every row is finite and every lse plausible (>= its diagonal score's log-sum)
     assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("peaky", [False, True])
+def test_long_context_workload_whole_tiles(cuda_device, peaky):
+    """Whole query tiles of the long-context workload, element by element:
+    for each of the 4 sequences the first, a middle and the last 128-row tile,
+    every one of the 32 query heads (both heads of every GQA pair a CTA runs,
+    the full span of ~256 key tiles with the lazy rescale, the causal diagonal
+    tile), against the oracle's block-of-rows entry."""
+    case = I.config5(peaky=peaky)
+    out, lse = run_prefill(case, cuda_device)
+    starts = np.concatenate([[0], np.cumsum(case.q_lens.numpy())])
+    for b in range(case.batch):
+        Q = int(case.q_lens[b])
+        n_qt = (Q + 127) // 128
+        for qt in sorted({0, n_qt // 2, n_qt - 1}):
+            i0, i1 = qt * 128, min(qt * 128 + 128, Q)
+            ro, rl = oracle.paged_prefill_tile(case.q, case.k_new, case.v_new, case.k_cache,
+                                               case.v_cache, case.block_tables, case.ctx_lens,
+                                               case.q_lens, case.scale, case.mask_kind, b, i0, i1)
+            go = out[starts[b] + i0:starts[b] + i1]
+            gl = lse[starts[b] + i0:starts[b] + i1]
+            assert_attention_close(go, gl, ro, rl, torch.bfloat16,
+                                   f"{case.name} b{b} tile{qt} peaky={peaky}")
 
 
 def test_decode_equals_last_row_of_prefill(cuda_device):

@@ -188,52 +188,3 @@ def test_two_calls_in_a_row_share_a_workspace(cuda_device):
     assert torch.equal(res[0][1], res[1][1])
     ref_o, ref_l = oracle_decode(case, case.k_cache, case.v_cache)
     assert_attention_close(res[1][0].cpu(), res[1][1].cpu(), ref_o, ref_l, case.dtype, "twice")
-
-
-_TC_CHILD = r"""
-import sys
-sys.path[:0] = [{root!r}, {tests!r}]
-import numpy as np
-import torch
-import paged_kv_cache_gather_b200 as pkv
-from paged_kv_cache_gather_b200 import inputs as I
-from parity import assert_attention_close, oracle_decode, to_dev, mask_of
-dev = torch.device("cuda:0")
-cases = [
-    I.config4(groups=2, beams=4, prefix=512, suffix=64, num_blocks=512, peaky=True),
-    I.make_shared_prefix_case("tc_ragged", seed=11, group_sizes=[3, 1, 2],
-                              prefix_lens=[40, 0, 32], suffix_lens=[5, 0, 17, 1, 9, 0],
-                              num_q_heads=8, num_kv_heads=2),
-    I.make_shared_prefix_case("tc_g32", seed=3, group_sizes=[32, 5], prefix_lens=[1000, 333],
-                              suffix_lens=list(range(37)), peaky=True),
-    I.make_shared_prefix_case("tc_bs8", seed=28, group_sizes=[4, 2], prefix_lens=[29, 16],
-                              suffix_lens=[1, 8, 19, 0, 7, 9], block_size=8, peaky=True),
-]
-for case in cases:
-    t = to_dev(case, dev)
-    err = torch.zeros(1, dtype=torch.int32, device=dev)
-    out, lse = pkv.paged_attention_decode_shared_prefix(
-        t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["seq_lens"],
-        case.extra["group_start"].to(dev), case.extra["shared_len"].to(dev),
-        case.extra["max_group_size"], case.scale, mask_of(case, t), dbg_err=err)
-    torch.cuda.synchronize()
-    pkv.read_dbg(err)
-    ref_o, ref_l = oracle_decode(case, case.k_cache, case.v_cache)
-    assert_attention_close(out.cpu(), lse.cpu(), ref_o, ref_l, case.dtype, case.name)
-print("ok")
-"""
-
-
-def test_tensor_core_variant_in_a_child_process(cuda_device):
-    # the kernel choice is read once per process: run the tensor-core variant's
-    # parity cases in a child with it selected
-    import os
-    import subprocess
-    import sys
-
-    tests = os.path.dirname(os.path.abspath(__file__))
-    root = os.path.dirname(tests)
-    env = dict(os.environ, PKV_GROUPED_TC="1")
-    r = subprocess.run([sys.executable, "-c", _TC_CHILD.format(root=root, tests=tests)],
-                       env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:] + r.stderr[-3000:]

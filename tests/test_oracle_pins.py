@@ -609,3 +609,41 @@ def test_planted_mask_mistakes_are_caught(monkeypatch, mutation):
                 worst = max(worst, float(np.max(np.abs(out[start + i, h] - o_ref))))
         start += ql[b]
     assert worst > 1e-6, f"mutation {mutation} went unnoticed"
+
+
+@pytest.mark.parametrize("kind,w,wph", [(A.MASK_NONE, 0, None), (A.MASK_CAUSAL, 0, None),
+                                        (A.MASK_SLIDING, 7, None),
+                                        (A.MASK_SLIDING, 0, [3, 0, 9, 1])])
+def test_prefill_tile_matches_brute_force(kind, w, wph):
+    """The tile entry (a block of query rows of one sequence, some heads) is the
+    same definition evaluated on a block: checked against the scalar brute
+    force over tiles that start mid-sequence and one cut by the chunk end."""
+    B, Hq, Hkv, d, bs = 2, 4, 2, 8, 4
+    ctx, ql = [9, 22], [7, 13]
+    gen = torch.Generator().manual_seed(17)
+    q, kc, vc, tab, _, scale = tiny_case(17, B, Hq, Hkv, d, bs, 40,
+                                         [c + n for c, n in zip(ctx, ql)], kind, w)
+    T = sum(ql)
+    qp = torch.randn(T, Hq, d, generator=gen, dtype=torch.float64)
+    kn = torch.randn(T, Hkv, d, generator=gen, dtype=torch.float64)
+    vn = torch.randn(T, Hkv, d, generator=gen, dtype=torch.float64)
+    kl, vl = kc.tolist(), vc.tolist()
+    g = Hq // Hkv
+    starts = [0, ql[0]]
+    for b, i0, i1, heads in [(0, 0, 7, None), (1, 4, 11, [3, 0]), (1, 10, 20, [1])]:
+        out, lse = oracle.paged_prefill_tile(qp, kn, vn, kc, vc, tab, ctx, ql, scale, kind, b,
+                                             i0, i1, heads=heads, window=w,
+                                             window_per_head=wph)
+        hs = list(range(Hq)) if heads is None else heads
+        rows = range(i0, min(i1, ql[b]))
+        assert out.shape == (len(rows), len(hs), d)
+        for r, i in enumerate(rows):
+            for j, h in enumerate(hs):
+                s0 = starts[b]
+                ek = [kn[s0 + t, h // g].tolist() for t in range(ql[b])]
+                ev = [vn[s0 + t, h // g].tolist() for t in range(ql[b])]
+                o_ref, l_ref = brute_paged_attention(
+                    qp[s0 + i, h].tolist(), kl, vl, tab[b].tolist(), ctx[b], ctx[b] + i, h // g,
+                    scale, kind, wph[h] if wph else w, ek, ev)
+                np.testing.assert_allclose(out[r, j], o_ref, rtol=0, atol=1e-13)
+                assert abs(lse[r, j] - l_ref) < 1e-13
