@@ -61,8 +61,10 @@ def peaks():
 # kernels are profiled again.
 PROFILED_TRAFFIC = {
     "decode": {"sources": ['csrc/decode.cu', 'csrc/pkv_common.cuh'],
-               "code_sha256": "f87eca92834f355213fdd1e53f086b5fa3bb0f33c46c8ad5180dda7d33d415b3",
-               "per_unit": 194071808 / 190134992,  # per algorithmic byte (16-seq ragged case)
+               "code_sha256": "109025c88ede4d20705278db577743c66e8d5702e992bc002e43b9e5ab5e075b",
+               # per algorithmic byte: one launch on the full ragged batch (862451200 B
+               # read + 4088064 B written for 860387680 algorithmic bytes)
+               "per_unit": (862451200 + 4088064) / 860387680,
                },
     "prefill": {"sources": ['csrc/prefill.cu', 'csrc/pkv_common.cuh', 'csrc/tc_sm100.cuh'],
                 "code_sha256": "b082f2e11624b3fc4976dd311201411e6ae21473f26a430a7fe378f8cd6012a8",
