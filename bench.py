@@ -250,11 +250,12 @@ class DecodeWork:
         vis = visible_tokens(lens.numpy(), c.window_per_seq.numpy())  # [steps, B]
         self.kv_bytes = vis.sum(axis=1) * Hkv * D * 2 * 2  # K and V, bf16
         self.io_bytes = B * Hq * D * 2 * 2 + B * Hq * 4 + ((vis + 15) // 16).sum(1) * Hkv * 4
-        self.append_bytes = B * Hkv * D * 2 * 2 * 2 + B * 8
+        self.append_bytes = B * Hkv * D * 2 * 2 * 2  # new K and V rows read and written
         # end-to-end steps: one host->device copy of every input of a step (packed
         # into one pinned buffer per step) and one device->host copy of out + lse
+        # (the fused call finds each new token's slot from the table: no slots)
         parts = [("q", self.q_h[0]), ("kn", self.kn_h[0]), ("vn", self.vn_h[0]),
-                 ("lens", self.lens_h[0]), ("slots", self.slots_h[0]), ("tab", self.tab_h)]
+                 ("lens", self.lens_h[0]), ("tab", self.tab_h)]
         self.layout, off = {}, 0
         for name, t in parts:
             nbytes = t.numel() * t.element_size()
@@ -263,8 +264,7 @@ class DecodeWork:
         self.pack_h = torch.empty(steps, off, dtype=torch.uint8).pin_memory()
         for st in range(steps):
             for name, t in (("q", self.q_h[st]), ("kn", self.kn_h[st]), ("vn", self.vn_h[st]),
-                            ("lens", self.lens_h[st]), ("slots", self.slots_h[st]),
-                            ("tab", self.tab_h)):
+                            ("lens", self.lens_h[st]), ("tab", self.tab_h)):
                 o, nb, _, _ = self.layout[name]
                 self.pack_h[st, o:o + nb] = t.contiguous().view(torch.uint8).view(-1)
         # two device copies of the packed inputs and of the packed results, so
@@ -283,6 +283,14 @@ class DecodeWork:
         self.h2d = self.pack_h.shape[1]   # bytes actually copied per step (with alignment pads)
         self.d2h = rb
 
+    def step(self, s):
+        """One decode step in one call: append each sequence's new token at its
+        next position and decode (the fused entry point)."""
+        self.pkv.paged_attention_decode_append(self.q[s], self.kn[s], self.vn[s], self.k_cache,
+                                               self.v_cache, self.tab, self.lens[s],
+                                               self.case.scale, self.mask, out=self.out,
+                                               lse=self.lse, workspace=self.ws)
+
     def append(self, s):
         self.pkv.paged_kv_append(self.kn[s], self.vn[s], self.slots[s], self.k_cache, self.v_cache)
 
@@ -297,13 +305,41 @@ class DecodeWork:
 
     def e2e_run(self, s, b):
         v = self.views[b]
-        self.pkv.paged_kv_append(v["kn"], v["vn"], v["slots"], self.k_cache, self.v_cache)
-        self.pkv.paged_attention_decode(v["q"], self.k_cache, self.v_cache, v["tab"], v["lens"],
-                                        self.case.scale, self.mask, out=self.out_e[b],
-                                        lse=self.lse_e[b], workspace=self.ws)
+        self.pkv.paged_attention_decode_append(v["q"], v["kn"], v["vn"], self.k_cache,
+                                               self.v_cache, v["tab"], v["lens"], self.case.scale,
+                                               self.mask, out=self.out_e[b], lse=self.lse_e[b],
+                                               workspace=self.ws)
 
     def e2e_out(self, b):
         self.res_h[b].copy_(self.res_d[b], non_blocking=True)
+
+
+def two_call_steps(dw, pw, step_ids, stream):
+    """The same decode steps as two calls (paged_kv_append, then
+    paged_attention_decode), for comparison with the fused call, interleaved
+    with the prefill steps as in the timed region (so L2 starts each decode
+    step in the same state); rewrites the same slots with the same values, so
+    the caches end as before."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    a, b, c = [ev() for _ in step_ids], [ev() for _ in step_ids], [ev() for _ in step_ids]
+    torch.cuda.synchronize()
+    for i, s in enumerate(step_ids):
+        a[i].record(stream)
+        dw.append(s)
+        b[i].record(stream)
+        dw.decode(s)
+        c[i].record(stream)
+        if pw:
+            pw.append()
+            pw.prefill()
+    torch.cuda.synchronize()
+    n = len(step_ids)
+    app = sum(a[i].elapsed_time(b[i]) for i in range(n)) / n
+    dec = sum(b[i].elapsed_time(c[i]) for i in range(n)) / n
+    kv = float(sum(dw.kv_bytes[s] for s in step_ids)) / n
+    return {"append_ms": round(app, 4), "decode_ms": round(dec, 4),
+            "ms_per_step": round(app + dec, 4),
+            "kv_GBps": round(kv / ((app + dec) * 1e-3) / 1e9, 1)}
 
 
 class PrefillWork:
@@ -937,8 +973,7 @@ def main():
     # ---------------- device-timed region
     for s in range(args.warmup):
         if dw:
-            dw.append(s)
-            dw.decode(s)
+            dw.step(s)
         if pw:
             pw.append()
             pw.prefill()
@@ -958,10 +993,8 @@ def main():
         s = args.warmup + i
         if dw:
             d0[i].record(stream)
-            dw.append(s)
+            dw.step(s)
             d1[i].record(stream)
-            dw.decode(s)
-            d2[i].record(stream)
         if pw:
             p0[i].record(stream)
             pw.append()
@@ -989,25 +1022,23 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic"}
     launches = 0
     if dw:
-        dec_ms = [d1[i].elapsed_time(d2[i]) for i in range(n)]
-        app_ms = [d0[i].elapsed_time(d1[i]) for i in range(n)]
+        step_ms = [d0[i].elapsed_time(d1[i]) for i in range(n)]
         steps_idx = range(args.warmup, args.warmup + n)
         kv = float(sum(dw.kv_bytes[s] for s in steps_idx))
-        io = float(sum(dw.io_bytes[s] for s in steps_idx))
-        dec_total_ms = max_over_ranks(sum(dec_ms) + sum(app_ms), ws, dev)
-        dec_only_ms = max_over_ranks(sum(dec_ms), ws, dev)
-        # whole-job KV throughput of the decode steps (append + decode), all ranks
+        io = float(sum(dw.io_bytes[s] for s in steps_idx)) + n * dw.append_bytes
+        dec_total_ms = max_over_ranks(sum(step_ms), ws, dev)
+        # whole-job KV throughput of the decode steps (append fused into the
+        # decode launch), all ranks
         value = kv * ws / (dec_total_ms * 1e-3) / 1e9
-        achieved = (kv + io) / n / (dec_only_ms / n * 1e-3) / 1e9
+        achieved = (kv + io) / n / (dec_total_ms / n * 1e-3) / 1e9
         e2e_ms = max_over_ranks(e2e_dec_ms, ws, dev)
         line.update({
             "value": round(value, 2), "unit": "GB/s",
             "decode": {"ms_per_step": round(dec_total_ms / n, 4),
-                       "decode_ms": round(dec_only_ms / n, 4),
-                       "append_ms": round(sum(app_ms) / n, 4),
+                       "call": "paged_attention_decode_append (append fused in the decode launch)",
                        "kv_bytes_per_step": int(kv / n),
                        "tokens_visible_per_step": int(kv / n / (8 * 128 * 4))},
-            "roofline": {"kernel": "paged_attention_decode (main + combine)", "bound": "hbm",
+            "roofline": {"kernel": "paged_attention_decode_append (main + merge)", "bound": "hbm",
                          "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": round(achieved / pk["hbm_gbs"], 4),
                          "peak_kind": pk_kind,
@@ -1016,7 +1047,7 @@ def main():
             "e2e": {"value": round(kv * ws / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": int(dw.h2d), "d2h_bytes_per_step": int(dw.d2h)},
         })
-        launches += 3 * n
+        launches += 2 * n
     if pw:
         pre_ms = [p1[i].elapsed_time(p2[i]) for i in range(n)]
         papp_ms = [p0[i].elapsed_time(p1[i]) for i in range(n)]
@@ -1047,6 +1078,8 @@ def main():
     line["gpu_launches"] = launches
     line["config"] = workload_config(pw is not None, ws)
     line["clocks"] = clk
+    if rank == 0 and not args.no_extras and want_decode:
+        line["decode"]["two_calls"] = two_call_steps(dw, pw, step_ids, stream)
     if rank == 0 and not args.no_extras and not args.small and want_decode:
         flush = l2_flush_buffer(dev)
         line["decode_sweep_batch1"] = decode_sweep(dev, flush)

@@ -300,6 +300,32 @@ PKV_API int paged_attention_decode(const void* q, const void* k_cache, const voi
                            int32_t* dbg_err, void* stream);
 
 /*
+ * paged_attention_decode_append — one decode step in one launch: each
+ * sequence's new token is appended to the cache and the step's queries attend
+ * to the cache including it. Source: "Ultimate Guide to PagedAttention",
+ * dynamic growth (a generated token's K/V go into the next position of the
+ * sequence's blocks, no existing data moves) followed by the decode of
+ * "Paged Attention Meets FlexAttention".
+ *   k_new, v_new  [batch, num_kv_heads, head_dim] BF16: the token at position
+ *                 seq_lens[b]-1 of sequence b (seq_lens include it, as for
+ *                 paged_attention_decode); it is written, for every KV head,
+ *                 to block block_tables[b][(seq_lens[b]-1) / block_size], row
+ *                 (seq_lens[b]-1) % block_size of both pools (the block must
+ *                 already be in the table). Sequences with seq_lens[b] = 0
+ *                 append nothing.
+ * The pools and every result are bit-identical to paged_kv_append with those
+ * slots followed by paged_attention_decode with the same arguments. Other
+ * arguments, limits and errors as paged_attention_decode; BF16 pools only.
+ */
+PKV_API int paged_attention_decode_append(const void* q, const void* k_new, const void* v_new,
+                                          void* k_cache, void* v_cache, pkv_cache_desc cache,
+                                          const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                          const int32_t* seq_lens, int32_t batch,
+                                          int32_t num_q_heads, float scale, pkv_mask_mod mask,
+                                          void* out, float* lse, void* workspace,
+                                          size_t workspace_bytes, int32_t* dbg_err, void* stream);
+
+/*
  * paged_attention_decode_fp8 — paged_attention_decode over E4M3 pools written
  * by paged_kv_append_fp8 (half the bytes of bf16 per token). Same arguments,
  * layouts, results and errors as paged_attention_decode, plus the row scales

@@ -31,6 +31,7 @@ from .ops import (  # noqa: F401
     document,
     no_mask,
     paged_attention_decode,
+    paged_attention_decode_append,
     paged_attention_decode_fp8,
     paged_attention_decode_shared_prefix,
     paged_attention_prefill,

@@ -51,6 +51,7 @@ EXPORTS = (
     "paged_kv_copy_blocks_fp8",
     "paged_attention_decode_workspace_size",
     "paged_attention_decode",
+    "paged_attention_decode_append",
     "paged_attention_prefill",
     "paged_attention_decode_noalloc",
     "paged_attention_decode_shared_prefix_workspace_size",
@@ -111,6 +112,10 @@ def _declare(lib):
     lib.paged_attention_decode.argtypes = [_vp, _vp, _vp, CacheDescC, _vp, _i32, _vp, _i32, _i32,
                                            _f32, MaskModC, _vp, _vp, _vp, _sz, _vp, _vp]
     lib.paged_attention_decode.restype = ctypes.c_int
+    lib.paged_attention_decode_append.argtypes = [_vp, _vp, _vp, _vp, _vp, CacheDescC, _vp, _i32,
+                                                  _vp, _i32, _i32, _f32, MaskModC, _vp, _vp, _vp,
+                                                  _sz, _vp, _vp]
+    lib.paged_attention_decode_append.restype = ctypes.c_int
     lib.paged_attention_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, CacheDescC, _vp, _i32, _vp,
                                             _vp, _i32, _i32, _i32, _f32, MaskModC, _vp, _vp, _vp,
                                             _vp]

@@ -239,7 +239,8 @@ size_t paged_attention_decode_workspace_size(int32_t batch, int32_t num_q_heads,
 }
 
 static int decode_entry(const char* fn, const void* q, const void* k_cache, const void* v_cache,
-                        const float* k_scale, const float* v_scale, pkv_cache_desc cache,
+                        const float* k_scale, const float* v_scale, const void* k_new,
+                        const void* v_new, pkv_cache_desc cache,
                         const int32_t* block_tables, int32_t max_blocks_per_seq,
                         const int32_t* seq_lens, int32_t batch, int32_t num_q_heads, float scale,
                         pkv_mask_mod mask, void* out, float* lse, void* workspace,
@@ -263,7 +264,8 @@ static int decode_entry(const char* fn, const void* q, const void* k_cache, cons
       (fp8 && (!k_scale || !v_scale)))
     return fail(PKV_ERR_INVALID_ARG, "%s: null pointer", fn);
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
-      !aligned16(workspace) || (fp8 && (!aligned16(k_scale) || !aligned16(v_scale))))
+      !aligned16(workspace) || (fp8 && (!aligned16(k_scale) || !aligned16(v_scale))) ||
+      !aligned16(k_new) || !aligned16(v_new))
     return fail(PKV_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", fn);
   const size_t need = decode_workspace_size(batch, num_q_heads, cache);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need))
@@ -274,6 +276,8 @@ static int decode_entry(const char* fn, const void* q, const void* k_cache, cons
                lse,       workspace, workspace_bytes, dbg_err, static_cast<cudaStream_t>(stream)};
   a.k_scale = k_scale;
   a.v_scale = v_scale;
+  a.k_new = k_new;
+  a.v_new = v_new;
   return launch_decode(a);
 }
 
@@ -283,7 +287,8 @@ int paged_attention_decode(const void* q, const void* k_cache, const void* v_cac
                            int32_t num_q_heads, float scale, pkv_mask_mod mask, void* out,
                            float* lse, void* workspace, size_t workspace_bytes,
                            int32_t* dbg_err, void* stream) {
-  return decode_entry("paged_attention_decode", q, k_cache, v_cache, nullptr, nullptr, cache,
+  return decode_entry("paged_attention_decode", q, k_cache, v_cache, nullptr, nullptr, nullptr,
+                      nullptr, cache,
                       block_tables, max_blocks_per_seq, seq_lens, batch, num_q_heads, scale, mask,
                       out, lse, workspace, workspace_bytes, dbg_err, stream);
 }
@@ -300,9 +305,28 @@ int paged_attention_decode_fp8(const void* q, const void* k_cache, const void* v
     g_last_error[0] = 0;
     return fail(PKV_ERR_INVALID_ARG, "%s: the pool must be E4M3", fn);
   }
-  return decode_entry(fn, q, k_cache, v_cache, k_scale, v_scale, cache, block_tables,
+  return decode_entry(fn, q, k_cache, v_cache, k_scale, v_scale, nullptr, nullptr, cache,
+                      block_tables,
                       max_blocks_per_seq, seq_lens, batch, num_q_heads, scale, mask, out, lse,
                       workspace, workspace_bytes, dbg_err, stream);
+}
+
+int paged_attention_decode_append(const void* q, const void* k_new, const void* v_new,
+                                  void* k_cache, void* v_cache, pkv_cache_desc cache,
+                                  const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t* seq_lens, int32_t batch, int32_t num_q_heads,
+                                  float scale, pkv_mask_mod mask, void* out, float* lse,
+                                  void* workspace, size_t workspace_bytes, int32_t* dbg_err,
+                                  void* stream) {
+  const char* fn = "paged_attention_decode_append";
+  g_last_error[0] = 0;
+  if (int st = check_cache(cache, fn)) return st;
+  if (cache.dtype != PKV_BF16)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: bf16 pools only", fn);
+  if (batch > 0 && (!k_new || !v_new)) return fail(PKV_ERR_INVALID_ARG, "%s: null pointer", fn);
+  return decode_entry(fn, q, k_cache, v_cache, nullptr, nullptr, k_new, v_new, cache,
+                      block_tables, max_blocks_per_seq, seq_lens, batch, num_q_heads, scale, mask,
+                      out, lse, workspace, workspace_bytes, dbg_err, stream);
 }
 
 int paged_kv_append_fp8(const void* k, const void* v, const int64_t* slot_mapping,

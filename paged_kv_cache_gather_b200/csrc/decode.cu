@@ -54,6 +54,12 @@ struct DecodeParams {
   pkv_mask_mod mask;
   const float* k_scale;  // E4M3 pools: float32 scale of each stored row [pool rows]
   const float* v_scale;
+  // fused append: each sequence's newest token [batch, num_kv_heads, D], written
+  // into the pools at position seq_lens[b]-1 of its block table
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  __nv_bfloat16* k_pool;
+  __nv_bfloat16* v_pool;
   __nv_bfloat16* out;
   float* lse;
   float* ws_o;         // [2 * workers, group, D] partial outputs (normalised)
@@ -194,7 +200,13 @@ struct Cfg {
 // decoded to f16 exactly (cvt.rn.f16x2.e4m3x2) and the MMAs run in f16: K's
 // row scales multiply the scores, V's row scales (times 256, which keeps the
 // products clear of f16 subnormals and is divided out at the end) multiply P.
-template <int D, int NSTAGE, int WPC, bool PH, bool KV8>
+// APPEND: the decode step's append is fused in. The worker that holds the last
+// tile of a (sequence, KV head) segment writes that sequence's new token
+// (k_new/v_new) into the pools at position seq_lens[b]-1 of its block table
+// and into the tile it has just loaded, over the row the pool held before; no
+// other worker reads that row, so the result is that of an append followed by
+// a decode.
+template <int D, int NSTAGE, int WPC, bool PH, bool KV8, bool APPEND = false>
 __global__ void __launch_bounds__(WPC * 32, 1)
     decode_bf16_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
@@ -385,6 +397,33 @@ __global__ void __launch_bounds__(WPC * 32, 1)
     }
     const int tok0 = (cur.s.t0 + (int)(cur.t - cur.seg_first)) * kTile;
     const bool partial = tok0 < cur.s.lo || tok0 + kTile > cur.s.hi;
+    if constexpr (APPEND) {
+      const int last = cur.s.hi - 1;  // the new token's position
+      if (last >= tok0 && last < tok0 + kTile) {
+        // 16-byte chunks of the new K row (lanes 0..D/8-1) and V row (the next D/8)
+        constexpr int kChunks = D / 8;
+        const int r = last - tok0;
+        if (lane < 2 * kChunks) {
+          const bool isv = lane >= kChunks;
+          const int ch = isv ? lane - kChunks : lane;
+          const int64_t src = ((int64_t)cur.b * p.num_kv_heads + cur.kvh) * D;
+          const uint4 val =
+              __ldg(reinterpret_cast<const uint4*>((isv ? p.v_new : p.k_new) + src) + ch);
+          *reinterpret_cast<uint4*>(kst + (isv ? C::kTileBytes : 0) + (ch >> 3) * (kTile * 128) +
+                                    r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = val;
+          const int j = last >> p.bs_shift;
+          const int blk = j < p.max_blocks ? __ldg(p.tables + (int64_t)cur.b * p.max_blocks + j) : -1;
+          if (blk >= 0 && blk < p.num_blocks) {
+            const int64_t grow = ((int64_t)(blk * p.num_kv_heads + cur.kvh) << p.bs_shift) +
+                                 (last & bs_mask);
+            *(reinterpret_cast<uint4*>((isv ? p.v_pool : p.k_pool) + grow * D) + ch) = val;
+          }  // an invalid id was flagged when the tile was loaded
+        }
+        // these generic writes precede the next TMA write of this stage
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+    }
     if constexpr (KV8) {
       // decode the V codes into the f16 work tile (row r, 16-code chunks
       // (lane & 1) * 4 ..); rows outside [lo, hi) become zero
@@ -820,7 +859,7 @@ __global__ void __launch_bounds__(128) decode_f32_kernel(
 
 namespace {
 
-template <int D, int NSTAGE, int WPC, bool PH, bool KV8 = false>
+template <int D, int NSTAGE, int WPC, bool PH, bool KV8 = false, bool APPEND = false>
 int launch_bf16_impl(const DecodeArgs& a) {
   using Cf = Cfg<D, KV8>;
   const int sms = device_sm_count();
@@ -833,7 +872,7 @@ int launch_bf16_impl(const DecodeArgs& a) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(decode_bf16_kernel<D, NSTAGE, WPC, PH, KV8>,
+    if (cudaFuncSetAttribute(decode_bf16_kernel<D, NSTAGE, WPC, PH, KV8, APPEND>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return check_launch("paged_attention_decode: smem attribute");
     attr_set[dev] = true;
@@ -864,6 +903,10 @@ int launch_bf16_impl(const DecodeArgs& a) {
   p.mask = a.mask;
   p.k_scale = a.k_scale;
   p.v_scale = a.v_scale;
+  p.k_new = static_cast<const __nv_bfloat16*>(a.k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(a.v_new);
+  p.k_pool = static_cast<__nv_bfloat16*>(const_cast<void*>(a.k_cache));
+  p.v_pool = static_cast<__nv_bfloat16*>(const_cast<void*>(a.v_cache));
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.lse = a.lse;
   const size_t o_bytes = (size_t)2 * workers * g * D * 4;
@@ -874,7 +917,8 @@ int launch_bf16_impl(const DecodeArgs& a) {
   p.workers = workers;
   p.dbg = a.dbg;
 
-  decode_bf16_kernel<D, NSTAGE, WPC, PH, KV8><<<sms, WPC * 32, smem, a.stream>>>(kmap, vmap, p);
+  decode_bf16_kernel<D, NSTAGE, WPC, PH, KV8, APPEND><<<sms, WPC * 32, smem, a.stream>>>(kmap, vmap,
+                                                                                         p);
   if (int st = check_launch("paged_attention_decode")) return st;
   const int64_t items = (int64_t)a.batch * a.cache.num_kv_heads * g;
   cudaLaunchConfig_t cfg = {};
@@ -904,6 +948,10 @@ int launch_bf16(const DecodeArgs& a) {
       if (per_head) return launch_bf16_impl<D, 3, 12, true, true>(a);
       return launch_bf16_impl<D, 2, 16, false, true>(a);
     }
+  }
+  if (a.k_new) {
+    if (per_head) return launch_bf16_impl<D, (D == 128 ? 2 : 4), 12, true, false, true>(a);
+    return launch_bf16_impl<D, (D == 128 ? 2 : 4), 12, false, false, true>(a);
   }
   if (per_head) return launch_bf16_impl<D, (D == 128 ? 2 : 4), 12, true>(a);
   return launch_bf16_impl<D, (D == 128 ? 2 : 4), 12, false>(a);

@@ -76,6 +76,9 @@ struct DecodeArgs {
   cudaStream_t stream;
   const float* k_scale = nullptr;  // E4M3 pools: row scales [num_blocks * Hkv * block_size]
   const float* v_scale = nullptr;
+  // fused append (bf16 pools): newest token of each sequence [batch, Hkv, head_dim]
+  const void* k_new = nullptr;
+  const void* v_new = nullptr;
 };
 
 size_t decode_workspace_size(int32_t batch, int32_t num_q_heads, const pkv_cache_desc& c);

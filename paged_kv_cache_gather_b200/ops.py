@@ -297,6 +297,44 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, seq_lens, scale=No
     return out, lse
 
 
+def paged_attention_decode_append(q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens,
+                                  scale=None, mask_mod: Optional[MaskMod] = None, *, out=None,
+                                  lse=None, workspace=None, dbg_err=None):
+    """One decode step in one launch: sequence b's new token (k_new[b], v_new[b],
+    [B, Hkv, d]) is written at position seq_lens[b]-1 of its block table, then
+    the queries attend to the cache including it. Returns (out, lse)."""
+    _check_pool(k_cache, v_cache)
+    dev = k_cache.device
+    B, Hq, d = q.shape
+    _check(k_cache.dtype == torch.bfloat16, "bf16 pools only")
+    for t, name in ((k_new, "k_new"), (v_new, "v_new")):
+        _check(t.dtype == k_cache.dtype and t.device == dev and t.is_contiguous() and
+               tuple(t.shape) == (B, k_cache.shape[1], d),
+               f"{name} must be contiguous [B, num_kv_heads, head_dim] in the cache dtype")
+    _i32(block_tables, "block_tables", dev)
+    _i32(seq_lens, "seq_lens", dev)
+    _check(q.dtype == k_cache.dtype and q.device == dev and q.is_contiguous(),
+           "q must be contiguous, on the cache's device, in the cache dtype")
+    _check(d == k_cache.shape[3], "head_dim mismatch")
+    _check(block_tables.dim() == 2 and block_tables.shape[0] == B and seq_lens.numel() == B,
+           "block_tables [B, M] and seq_lens [B] must match q's batch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    mask_mod = mask_mod or no_mask()
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = decode_workspace(B, Hq, k_cache)
+    L.check(L.lib().paged_attention_decode_append(
+        _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), cache_desc(k_cache),
+        _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), B, Hq, float(scale),
+        mask_mod.to_c(B, dev, Hq), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _ptr(dbg_err), _stream()))
+    return out, lse
+
+
 def shared_prefix_workspace_size(batch, num_q_heads, k_cache):
     return int(L.lib().paged_attention_decode_shared_prefix_workspace_size(
         batch, num_q_heads, cache_desc(k_cache)))
