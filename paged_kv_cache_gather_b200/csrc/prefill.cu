@@ -13,13 +13,21 @@
 //    of query heads of that KV head's group, 128-row query tile); the two
 //    heads share every K/V tile the CTA loads (GQA). Units are handed out
 //    round-robin, longest (last query tiles) first.
-//  * Warp roles: warps 0-3 and 4-7 are the softmax warpgroups of head 0 and
-//    head 1 (one query row per thread); warp 8 issues TMA loads; warp 9
-//    allocates tensor memory and issues the MMAs.
+//  * Warp roles: warps 0-7 turn head 0's scores into probabilities, warps
+//    8-15 head 1's: two threads per query row, one per half of the 128 key
+//    columns (warps 0-3: keys 0-63, warps 4-7: keys 64-127), so each head's
+//    softmax runs on two warps per SM sub-partition and its exponentials
+//    keep the transcendental unit busy. The halves of a row trade their
+//    maxima through shared memory once per tile and their row sums once per
+//    unit, ordered by a named barrier of the head's 8 warps. Every tile
+//    starts with a vote (bar.red.and) on the head's bounded waits, so the 8
+//    warps leave together on a timeout and no barrier is left waiting. Warp
+//    16 issues TMA loads; warp 17 allocates tensor memory and issues the MMAs.
 //  * Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.
 //    S = Q K^T is written by tcgen05.mma (M=128, N=128 keys, K=16 x 8); the
-//    softmax warps read S, write P as bf16 into the first 64 columns of the
-//    same S region, and O += P V reads P straight from tensor memory
+//    softmax warps read S and write P as bf16 into the same S region (keys
+//    0-63 in columns 0-31, keys 64-127 in columns 64-95: each half of a row
+//    over its own columns), and O += P V reads P straight from tensor memory
 //    (A operand in TMEM) with V as an MN-major shared-memory operand.
 //  * MMA issue order S0(j), PV1(j-1), S1(j), PV0(j): while one warpgroup
 //    turns its S into P the tensor core runs the other head's work.
@@ -50,7 +58,9 @@ constexpr int kN = 128;             // keys per tile
 constexpr int kStages = 2;          // K/V ring depth
 constexpr int kTileBytes = kN * kD * 2;   // 32 KB (K or V or Q tile)
 constexpr int kHalfBytes = kTileBytes / 2;
-constexpr int kThreads = 320;       // softmax head 0 (4 warps), head 1 (4), TMA (1), MMA (1)
+constexpr int kThreads = 576;       // softmax head 0 (8 warps), head 1 (8), TMA (1), MMA (1)
+constexpr int kTmaWarp = 16;
+constexpr int kMmaWarp = 17;
 constexpr int kMaxBatch = 4096;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 
@@ -85,8 +95,10 @@ struct SmemLayout {
   static constexpr int kBars = kKV + kStages * 2 * kTileBytes;
   static constexpr int kNumBars = 2 + 4 * kStages + 9;
   static constexpr int kTmemSlot = kBars + kNumBars * 8;
-  static constexpr int kQoff = kTmemSlot + 16;  // int32 [batch + 1]
-  static constexpr int kMaxQt = kQoff - 8;      // int32 (placed before the prefix)
+  static constexpr int kMaxQt = kTmemSlot + 4;  // int32, then the abort flag
+  // one float per (head, half, parity, row): row maxima / sums traded by the halves
+  static constexpr int kXchg = (kTmemSlot + 16 + 15) & ~15;
+  static constexpr int kQoff = kXchg + 2 * 2 * 2 * kM * 4;  // int32 [batch + 1]
 };
 
 // barrier indices
@@ -103,6 +115,9 @@ enum : int {
   BAR_O_FREE = BAR_O_FULL + 2,     // + head
   BAR_V_FIXED = BAR_O_FREE + 2,    // a V tile whose rows past the context end were zeroed
 };
+
+// Named barriers (0 is __syncthreads): 1 + head for the 8 softmax warps of a head.
+constexpr int kHeadBarrier = 1;
 
 struct Unit {
   bool valid;
@@ -193,6 +208,24 @@ __device__ __forceinline__ bool wait_or_flag(uint32_t bar, uint32_t parity, int3
   return ok;
 }
 
+// Named barrier of `n` threads; the `and` form also returns whether `pred`
+// held in all of them (every arriving thread gets the same answer).
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ bool named_and(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -215,6 +248,8 @@ struct Maps {
   CUtensorMap vpool;
 };
 
+// 18 warps: five on two of the SM's four sub-partitions, whose 16K-register
+// files then allow at most 96 registers a thread
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ Maps maps, const PrefillParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -232,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* abort_flag = reinterpret_cast<int*>(smem + L::kMaxQt + 4);
 
   // ---- set-up: barriers, tensor memory, per-sequence query offsets
-  if (warp == 8) {
+  if (warp == kTmaWarp) {
     if (lane == 0) {
       mbar_init(bar(BAR_Q_FULL), 1);
       mbar_init(bar(BAR_Q_EMPTY), 1);
@@ -244,9 +279,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int h = 0; h < 2; ++h) {
         mbar_init(bar(BAR_S_FULL + h), 1);
-        mbar_init(bar(BAR_P_FULL + h), 128);
+        mbar_init(bar(BAR_P_FULL + h), 256);
         mbar_init(bar(BAR_O_FULL + h), 1);
-        mbar_init(bar(BAR_O_FREE + h), 128);
+        mbar_init(bar(BAR_O_FREE + h), 256);
       }
       mbar_init(bar(BAR_V_FIXED), 1);
       *abort_flag = 0;
@@ -279,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       *max_qt_s = mq;
       if (run != p.total_q && blockIdx.x == 0) flag_error(p.dbg, PKV_DBG_QLEN_SUM);
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     tc::tmem_alloc(smem_u32(tmem_slot), 512);
     tc::tmem_relinquish();
   }
@@ -291,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t num_units = (int64_t)max_qt * p.batch * p.num_kv_heads * p.pairs;
   const uint32_t q_bytes = (p.two_heads ? 2u : 1u) * kTileBytes;
 
-  if (warp == 8) {
+  if (warp == kTmaWarp) {
     // ================================================================ TMA producer
     const int nbox = kN / p.box_rows;  // paged boxes per context tile (8 or 16)
     const int bs_mask = (1 << p.bs_shift) - 1;
@@ -393,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       ++unit_k;
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
     const uint32_t idesc_s = tc::idesc_bf16(kM, kN, false, false);
     const uint32_t idesc_o = tc::idesc_bf16(kM, kD, false, true);
@@ -417,10 +452,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mma_ss(d, dq + off, dk + off, idesc_s, kk > 0);
       }
     };
+    // P of keys 0-63 sits in columns 0-31 of the head's S region, P of keys
+    // 64-127 in columns 64-95 (each softmax half packs its P over its own
+    // first 32 columns); a k-step of 16 keys reads 8 columns
     auto issue_pv = [&](uint32_t d, uint32_t p_tmem, uint64_t dv, bool acc) {
 #pragma unroll
       for (int kk = 0; kk < kN / 16; ++kk)
-        tc::mma_ts(d, p_tmem + kk * 8, dv + (uint64_t)(kk * (2048 >> 4)), idesc_o, acc || kk > 0);
+        tc::mma_ts(d, p_tmem + kk * 8 + (kk >= 4 ? 32 : 0), dv + (uint64_t)(kk * (2048 >> 4)),
+                   idesc_o, acc || kk > 0);
     };
     for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
       const Unit x = unit_of(p, qoff, max_qt, u);
@@ -509,13 +548,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       ++unit_k;
     }
-  } else if (warp < 8) {
+  } else if (warp < 16) {
     // ================================================================ softmax warpgroups
-    const int hsel = warp >> 2;              // which head of the pair
+    const int hsel = warp >> 3;              // which head of the pair
+    const int csel = (warp >> 2) & 1;        // which half of the key columns
     const int row = (warp & 3) * 32 + lane;  // query row of the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t S = tmem + hsel * 128 + lane_base;
-    const uint32_t O = tmem + 256 + hsel * 128 + lane_base;
+    const uint32_t S = tmem + hsel * 128 + csel * 64 + lane_base;       // this half's 64 scores
+    const uint32_t Pw = S;  // its 32 words of bf16 P go over its own first 32 columns
+    const uint32_t O = tmem + 256 + hsel * 128 + csel * 64 + lane_base; // its 64 output columns
+    float* xch = reinterpret_cast<float*>(smem + L::kXchg);
+    const int hbar = kHeadBarrier + hsel;
+    uint32_t x_cnt = 0;
+    // trade one float of this row with the other half of the head (slots
+    // alternate, so a slot is rewritten only after the head's next barrier,
+    // which the other half reaches after reading it)
+    auto exchange = [&](float mine) -> float {
+      const uint32_t par = x_cnt & 1;
+      xch[((hsel * 2 + csel) * 2 + par) * kM + row] = mine;
+      named_sync(hbar, 256);
+      ++x_cnt;
+      return xch[((hsel * 2 + (csel ^ 1)) * 2 + par) * kM + row];
+    };
     int unit_k = 0;
     uint32_t s_cnt = 0;
     for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
@@ -537,31 +591,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row_hi = mask_hi(p.mask, x.b, qpos, n_keys);
       const int lo_max = mask_lo(p.mask, x.b, h_own, qmax);
       const int hi_min = mask_hi(p.mask, x.b, qmin, n_keys);
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
       bool ok = true;
       for (int j = 0; j < n; ++j, ++s_cnt) {
-        if (!wait_or_flag(bar(BAR_S_FULL + hsel), s_cnt & 1, p.dbg, abort_flag, true)) { ok = false; break; }
+        ok = wait_or_flag(bar(BAR_S_FULL + hsel), s_cnt & 1, p.dbg, abort_flag, true);
+        if (!named_and(hbar, 256, ok)) { ok = false; break; }  // all 8 warps go on, or none
         tc::fence_after_sync();
         bool ctx;
         int idx, kp0;
         tile_of(x, j, ctx, idx, kp0);
         const int key_end = ctx ? x.C : n_keys;
         const bool full = kp0 + kN <= min(key_end, hi_min) && kp0 >= lo_max;
-        // pass 1: the whole S row of this thread in one tensor-memory round trip
+        // pass 1: this half's 64 scores, masked in tensor memory (masked keys
+        // become -inf, so pass 2 needs no mask), and their maximum
         float mx;
         {
-          uint32_t r[4][32];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tc::ld32(S + c * 32, r[c]);
+          uint32_t r[2][32];
+          tc::ld32(S, r[0]);
+          tc::ld32(S + 32, r[1]);
           tc::wait_ld();
           if (!full) {
-            // the visible keys of a row form one interval of columns [vlo, vhi);
-            // masked scores become -inf in tensor memory, so pass 2 needs no mask
-            const int vhi = min(kN, min(key_end, row_hi) - kp0);
-            const int vlo = max(0, row_lo - kp0);
+            // the visible keys of a row form one interval of columns [vlo, vhi)
+            const int c0 = kp0 + csel * 64;  // key of this half's first column
+            const int vhi = min(64, min(key_end, row_hi) - c0);
+            const int vlo = max(0, row_lo - c0);
             const uint32_t span = (uint32_t)max(vhi - vlo, 0);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
 #pragma unroll
               for (int i = 0; i < 32; ++i)
                 if ((uint32_t)(c * 32 + i - vlo) >= span) r[c][i] = __float_as_uint(-INFINITY);
@@ -569,17 +625,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc::wait_st();
           }
-          float mx4[4];
+          float a0 = -INFINITY, a1 = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float a0 = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < 32; i += 2)
-              a0 = fmax3(a0, __uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1]));
-            mx4[c] = a0;
+          for (int i = 0; i < 32; i += 2) {
+            a0 = fmax3(a0, __uint_as_float(r[0][i]), __uint_as_float(r[0][i + 1]));
+            a1 = fmax3(a1, __uint_as_float(r[1][i]), __uint_as_float(r[1][i + 1]));
           }
-          mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+          mx = fmaxf(a0, a1);
         }
+        mx = fmaxf(mx, exchange(mx));         // the row maximum, the same in both halves
         const float mxs = mx * p.scale_log2;  // scale > 0 keeps the order
         // lazy rescale: move the reference maximum only when it grows by > 2^8
         float alpha = 1.f;
@@ -588,45 +642,45 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = mxs;
         }
         const float mb = (m == -INFINITY) ? 0.f : m;
-        // pass 2: the row again in one round trip; P = exp2(s*c - m) (masked keys
-        // hold -inf and give 0) with the argument and the row sum on packed
-        // float pairs, packed in place to bf16 pairs (P[2k], P[2k+1] -> word k)
-        // and stored over the first 64 columns of S
+        // pass 2, 32 columns at a time: P = exp2(s*c - m) (masked keys hold
+        // -inf and give 0) with the argument and the row sum on packed float
+        // pairs, packed to bf16 pairs (P[2k], P[2k+1] -> word k) and stored
+        // over the first 32 of this half's own columns, so neither half
+        // writes where the other still reads
         float ls[8];
         {
-          uint32_t r[4][32];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tc::ld32(S + c * 32, r[c]);
-          tc::wait_ld();
           const uint64_t c2 = f2(p.scale_log2, p.scale_log2), nm2 = f2(-mb, -mb);
           uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+          uint32_t pw[32];
 #pragma unroll
-          for (int k = 0; k < 64; ++k) {
-            const int f0 = 2 * k, f1 = 2 * k + 1;
-            const uint64_t xv = ffma2(
-                f2(__uint_as_float(r[f0 >> 5][f0 & 31]), __uint_as_float(r[f1 >> 5][f1 & 31])),
-                c2, nm2);
-            float x0, x1;
-            f2_split(xv, x0, x1);
-            const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-            acc[k & 3] = fadd2(acc[k & 3], f2(e0, e1));
-            r[k >> 5][k & 31] = pack_bf16x2(e0, e1);
+          for (int c = 0; c < 2; ++c) {
+            uint32_t r[32];
+            tc::ld32(S + c * 32, r);
+            tc::wait_ld();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const uint64_t xv =
+                  ffma2(f2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), c2, nm2);
+              float x0, x1;
+              f2_split(xv, x0, x1);
+              const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+              acc[k & 3] = fadd2(acc[k & 3], f2(e0, e1));
+              pw[c * 16 + k] = pack_bf16x2(e0, e1);
+            }
           }
-          tc::st32(S, r[0]);
-          tc::st32(S + 32, r[1]);
+          tc::st32(Pw, pw);
 #pragma unroll
           for (int k = 0; k < 4; ++k) f2_split(acc[k], ls[2 * k], ls[2 * k + 1]);
         }
-        const float ls0 = (ls[0] + ls[1]) + (ls[2] + ls[3]);
-        const float ls1 = (ls[4] + ls[5]) + (ls[6] + ls[7]);
-        l = l * alpha + ls0 + ls1;
+        l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         // tcgen05.ld/st are warp-collective: the whole warp takes this branch
         // when any of its rows moved its maximum (the others scale by 1)
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          // rescale this row of O; the previous P*V has completed (it was issued
-          // before this S) and the next one waits for this thread's arrival
+          // rescale this half of the row of O; the previous P*V has completed
+          // (it was issued before this S) and the next one waits for this
+          // thread's arrival
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < 2; ++c) {
             uint32_t o[32];
             tc::ld32(O + c * 32, o);
             tc::wait_ld();
@@ -640,15 +694,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(BAR_P_FULL + hsel));
       }
       if (!ok) break;
-      // ---- epilogue: O / l -> bf16, lse
-      if (!wait_or_flag(bar(BAR_O_FULL + hsel), unit_k & 1, p.dbg, abort_flag, true)) break;
+      // ---- epilogue: O / l -> bf16 (each half its 64 columns), lse
+      ok = wait_or_flag(bar(BAR_O_FULL + hsel), unit_k & 1, p.dbg, abort_flag, true);
+      if (!named_and(hbar, 256, ok)) break;
       tc::fence_after_sync();
+      const float l_other = exchange(l);
+      const float lt = csel == 0 ? l + l_other : l_other + l;  // same order in both halves
       const int h = x.kvh * p.group + x.hp * (p.two_heads ? 2 : 1) + hsel;
       const bool valid_row = i_row < x.Q && x.qoff + i_row < p.total_q;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* dst = p.out + ((int64_t)(x.qoff + i_row) * p.num_q_heads + h) * kD;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      __nv_bfloat16* dst = p.out + ((int64_t)(x.qoff + i_row) * p.num_q_heads + h) * kD + csel * 64;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t o[32];
         tc::ld32(O + c * 32, o);
         tc::wait_ld();
@@ -664,9 +721,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (valid_row && p.lse)
+      if (csel == 0 && valid_row && p.lse)
         p.lse[(int64_t)(x.qoff + i_row) * p.num_q_heads + h] =
-            l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+            lt > 0.f ? (m + log2f(lt)) * kLn2 : -INFINITY;
       tc::fence_before_sync();
       mbar_arrive(bar(BAR_O_FREE + hsel));
       ++unit_k;
@@ -675,7 +732,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 512);
   }
