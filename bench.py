@@ -61,14 +61,16 @@ def peaks():
 # kernels are profiled again.
 PROFILED_TRAFFIC = {
     "decode": {"sources": ['csrc/decode.cu', 'csrc/pkv_common.cuh'],
-               "code_sha256": "109025c88ede4d20705278db577743c66e8d5702e992bc002e43b9e5ab5e075b",
-               # per algorithmic byte: one launch on the full ragged batch (862451200 B
-               # read + 4088064 B written for 860387680 algorithmic bytes)
-               "per_unit": (862451200 + 4088064) / 860387680,
+               "code_sha256": "87d8c0db844e94d0b5b686571bd31f0ac816443b959b3a751f7eae7df7d92e15",
+               # per algorithmic byte: one launch of the fused decode step on the full
+               # ragged batch (862712832 B read + 4083712 B written for 860911968 B)
+               "per_unit": (862712832 + 4083712) / 860911968,
                },
-    "prefill": {"sources": ['csrc/prefill.cu', 'csrc/pkv_common.cuh', 'csrc/tc_sm100.cuh'],
-                "code_sha256": "b082f2e11624b3fc4976dd311201411e6ae21473f26a430a7fe378f8cd6012a8",
-                "per_unit": 298716160 / 1065168666624,  # per causal FLOP (1-seq case)
+    "prefill": {"sources": ['csrc/prefill.cu', 'csrc/prefill_common.cuh', 'csrc/pkv_common.cuh',
+                            'csrc/tc_sm100.cuh'],
+                "code_sha256": "5a03e41c1b52e467e1f8bc793349c8c53fb0b298ac4840a4fddb1e350498b5e5",
+                # per causal FLOP: one launch on one long-context sequence
+                "per_unit": (165566976 + 12781568) / 1065168666624,
                 },
 }
 
