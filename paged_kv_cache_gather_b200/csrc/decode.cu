@@ -862,15 +862,7 @@ namespace {
 template <int D, int NSTAGE, int WPC, bool PH, bool KV8 = false, bool APPEND = false>
 int launch_bf16_impl(const DecodeArgs& a) {
   using Cf = Cfg<D, KV8>;
-  // one CTA per SM, fewer when the tables cannot hold enough 16-token tiles to
-  // give every worker kMinTilesPerWorker of them (small batches launch fewer CTAs)
-  int sms = device_sm_count();
-  {
-    const int64_t max_tiles = (int64_t)a.batch * a.cache.num_kv_heads *
-                              (((int64_t)a.max_blocks * a.cache.block_size + kTile - 1) / kTile);
-    const int64_t ctas = (max_tiles / kMinTilesPerWorker + WPC - 1) / WPC;
-    if (ctas < sms) sms = (int)(ctas < 1 ? 1 : ctas);
-  }
+  const int sms = device_sm_count();
   const int workers = sms * WPC;
   const int g = a.num_q_heads / a.cache.num_kv_heads;
   const size_t smem =
