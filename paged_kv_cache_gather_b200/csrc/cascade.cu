@@ -11,16 +11,18 @@
 // B200 design (bf16, head_dim 128):
 //  * One persistent launch of `grouped_decode_kernel` over a flat list of
 //    16-token tiles, as in the paged decode kernel. An item of the list is
-//    either a prefix item (one group, up to 32 query rows: every member's
-//    query heads of a KV head, row = member * g + head; keys: the group's
-//    shared prefix through its first member's block table) or an own-key item
+//    either a prefix item (one group, a block of up to 16 query rows, or 32
+//    when a KV head has more than 16 query heads: every member's query heads
+//    of a KV head, row = member * g + head; keys: the group's shared prefix
+//    through its first member's block table) or an own-key item
 //    (one sequence, its g query heads; keys from its shared length to its
 //    end). Each (item, KV head) segment is a run of tiles; warps take equal
 //    contiguous ranges of the whole list, so the work is balanced whatever the
 //    group sizes and lengths are.
-//  * The query rows of a segment are the N side of mma.sync m16n8k16 (four
-//    n-tiles of 8 rows), so a KV tile, loaded once by TMA into the warp's ring,
-//    serves all members of the group. S^T = K Q^T puts tokens on M; P^T is
+//  * The query rows of a segment are the N side of mma.sync m16n8k16 (two or
+//    four n-tiles of 8 rows), so a KV tile, loaded once by TMA into the warp's
+//    ring, serves all the segment's rows; a group's row blocks read the same
+//    prefix tiles, the later ones from L2. S^T = K Q^T puts tokens on M; P^T is
 //    transposed in registers (movmatrix) into the B operand of O^T += V^T P^T.
 //    The query tile of a segment is staged in the warp's shared memory
 //    (128-byte XOR swizzle) and read with ldmatrix. The path is HBM-bound: a
@@ -32,6 +34,7 @@
 //    (sequence, head) one warp that finds the sequence's group, merges the
 //    pieces of its prefix segment and of its own-key segment by log-sum-exp,
 //    merges the two, and writes bf16 out and the LSE.
+#include <algorithm>
 #include <climits>
 #include <cmath>
 
@@ -44,15 +47,21 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kTile = 16;            // tokens per tile
-constexpr int kRows = 32;            // query rows per segment (4 n-tiles of 8)
-constexpr int kNT = kRows / 8;
-constexpr int kWarps = 8;            // warps per CTA, one CTA per SM
+constexpr int kMaxRows = 32;         // query rows per segment at most (4 n-tiles of 8)
+// Rows per segment and warps per CTA (one CTA per SM). The kernel is
+// latency-bound: 16-row segments (168 registers) let 10 warps fit where 32-row
+// segments (252 registers) allowed 8, 94 us per call on the beams workload
+// against 111 us (11 warps: 97 us). Groups of more than 16 query heads per KV
+// head need 32-row segments.
+constexpr int kSmallRows = 16, kSmallWarps = 10;
+constexpr int kLargeRows = 32, kLargeWarps = 8;
+constexpr int kMaxWarps = kSmallWarps;
 constexpr int kStages = 2;           // TMA ring depth per warp
 constexpr int kMinTilesPerWorker = 2;
 constexpr int kTileBytes = kTile * kD * 2;            // K (or V) bytes of one tile
 constexpr int kStageBytes = 2 * kTileBytes;           // K then V
-constexpr int kQBytes = kRows * kD * 2;               // staged query rows of a segment
-constexpr int kWarpSmem = kStages * kStageBytes + kQBytes;
+// shared memory of one warp: its TMA ring and its segment's staged query rows
+__host__ __device__ constexpr int warp_smem(int rows) { return kStages * kStageBytes + rows * kD * 2; }
 
 struct GroupedParams {
   const __nv_bfloat16* q;      // [batch, Hq, D]
@@ -63,7 +72,8 @@ struct GroupedParams {
   const int32_t* shared_len;   // [batch]
   int32_t batch;
   int32_t num_groups;
-  int32_t row_blocks;          // prefix items per group: ceil(max_members * g / kRows)
+  int32_t seg_rows;            // query rows per segment (16 or 32)
+  int32_t row_blocks;          // prefix items per group: ceil(max_members * g / seg_rows)
   int32_t max_members;
   int32_t items;               // num_groups * row_blocks + batch
   int32_t num_kv_heads;
@@ -74,8 +84,8 @@ struct GroupedParams {
   float scale_log2;
   __nv_bfloat16* out;
   float* lse;
-  float* ws_o;                 // [2 * workers, kRows, D] pieces of split segments
-  float* ws_lse;               // [2 * workers, kRows]
+  float* ws_o;                 // [2 * workers, seg_rows, D] pieces of split segments
+  float* ws_lse;               // [2 * workers, seg_rows]
   float* whole_o;              // [2, batch * Hq, D]: prefix (0) / own keys (1), whole segments
   float* whole_lse;            // [2, batch * Hq]
   int32_t* ws_prefix;          // [items + 1] tiles per KV head before item i
@@ -114,7 +124,7 @@ __device__ __forceinline__ Item item_of(const GroupedParams& p, int i) {
     b0 = min(max(b0, 0), p.batch);
     b1 = min(max(b1, b0), min(p.batch, b0 + p.max_members));
     it.lead = b0;
-    it.rows = min(kRows, (b1 - b0) * p.group - it.rb * kRows);
+    it.rows = min(p.seg_rows, (b1 - b0) * p.group - it.rb * p.seg_rows);
     it.lo = 0;
     it.hi = it.rows > 0 ? clamp_len(p, __ldg(p.shared_len + b0)) : 0;
   } else {
@@ -218,7 +228,7 @@ __device__ __forceinline__ void cursor_advance(const GroupedParams& p, Cursor& c
 __device__ __forceinline__ void row_target(const GroupedParams& p, const Item& it, int kvh, int r,
                                            int& b, int& h) {
   if (it.prefix) {
-    const int R = it.rb * kRows + r;
+    const int R = it.rb * p.seg_rows + r;
     b = it.lead + R / p.group;
     h = kvh * p.group + R % p.group;
   } else {
@@ -235,9 +245,15 @@ __device__ __forceinline__ uint32_t swz(int rows, int r, int c) {
 
 }  // namespace
 
-__global__ void __launch_bounds__(kWarps * 32, 1)
+// NT: n-tiles of 8 query rows per segment; WARPS: warps per CTA.
+template <int NT, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 1)
     grouped_decode_kernel(const __grid_constant__ CUtensorMap kmap,
                           const __grid_constant__ CUtensorMap vmap, const GroupedParams p) {
+  constexpr int kNT = NT;
+  constexpr int kRows = NT * 8;
+  constexpr int kWarps = WARPS;
+  constexpr int kWarpSmem = warp_smem(kRows);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -587,7 +603,7 @@ __device__ __forceinline__ float segment_result(const GroupedParams& p, int lane
     float x = -INFINITY;
     if (w <= wl) {
       const int64_t sl = slot_of(w);
-      if (sl >= 0) x = __ldcg(p.ws_lse + sl * kRows + r);
+      if (sl >= 0) x = __ldcg(p.ws_lse + sl * p.seg_rows + r);
     }
     float mx = x;
 #pragma unroll
@@ -606,7 +622,7 @@ __device__ __forceinline__ float segment_result(const GroupedParams& p, int lane
     float wgt = 0.f;
     if (w <= wl) {
       sl = slot_of(w);
-      if (sl >= 0) wgt = __expf(__ldcg(p.ws_lse + sl * kRows + r) - lse);
+      if (sl >= 0) wgt = __expf(__ldcg(p.ws_lse + sl * p.seg_rows + r) - lse);
     }
     // eight pieces' loads in flight at a time (the loop is latency-bound)
     const int cnt = min(32, wl - base + 1);
@@ -620,7 +636,7 @@ __device__ __forceinline__ float segment_result(const GroupedParams& p, int lane
         const int64_t sj = __shfl_sync(0xffffffffu, sl, j & 31);
         const bool use = j < cnt && sj >= 0;
         wv[u] = use ? wj : 0.f;
-        v[u] = use ? __ldcg(reinterpret_cast<const float4*>(p.ws_o + (sj * kRows + r) * kD) +
+        v[u] = use ? __ldcg(reinterpret_cast<const float4*>(p.ws_o + (sj * p.seg_rows + r) * kD) +
                             lane)
                    : make_float4(0.f, 0.f, 0.f, 0.f);
       }
@@ -671,7 +687,7 @@ __global__ void __launch_bounds__(128) grouped_combine_kernel(const GroupedParam
     op[0] = op[1] = op[2] = op[3] = 0.f;
   } else {
     const int R = (b - b0) * p.group + hh;
-    lp = segment_result(p, lane, gi * p.row_blocks + R / kRows, kvh, R % kRows, row, op);
+    lp = segment_result(p, lane, gi * p.row_blocks + R / p.seg_rows, kvh, R % p.seg_rows, row, op);
   }
   const float ls = segment_result(p, lane, p.num_groups * p.row_blocks + b, kvh, hh,
                                   rows_all + row, os);
@@ -695,24 +711,47 @@ __global__ void __launch_bounds__(128) grouped_combine_kernel(const GroupedParam
 
 namespace {
 
-// Workspace: pieces (2 per worker), whole-segment results (prefix and own
-// keys per (sequence, head)), tile prefix over items (at most 5 * batch items:
-// groups * row blocks <= 4 * batch when max_group_size * g <= 128).
+// One launch of the main kernel with NT n-tiles of rows per segment and WARPS
+// warps per CTA (one CTA per SM).
+template <int NT, int WARPS>
+int launch_grouped(GroupedParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap, int sms,
+                   cudaStream_t s) {
+  const size_t smem = (size_t)WARPS * warp_smem(NT * 8) + WARPS * kStages * 8 + 1024;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(grouped_decode_kernel<NT, WARPS>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return check_launch("paged_attention_decode_shared_prefix: smem attribute");
+    attr_set[dev] = true;
+  }
+  p.workers = sms * WARPS;
+  grouped_decode_kernel<NT, WARPS><<<sms, WARPS * 32, smem, s>>>(kmap, vmap, p);
+  return check_launch("paged_attention_decode_shared_prefix");
+}
+
+// Workspace (sized for either segment shape): pieces (2 per worker),
+// whole-segment results (prefix and own keys per (sequence, head)), tile
+// prefix over items (at most 9 * batch items: groups * row blocks <= 8 * batch
+// when max_group_size * g <= 128 and segments hold 16 rows).
 struct Layout {
   size_t ws_o, ws_lse, whole_o, whole_lse, prefix, total;
 };
 
 Layout layout(int32_t batch, int32_t num_q_heads) {
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-  const size_t workers = (size_t)device_sm_count() * kWarps;
+  const size_t sms = (size_t)device_sm_count();
+  const size_t piece_rows =  // worker slots x rows per slot, the larger of the two shapes
+      std::max(sms * kSmallWarps * kSmallRows, sms * kLargeWarps * kLargeRows);
   const size_t rows = (size_t)batch * num_q_heads;
   Layout l;
   l.ws_o = 0;
-  l.ws_lse = l.ws_o + up(2 * workers * kRows * kD * 4);
-  l.whole_o = l.ws_lse + up(2 * workers * kRows * 4);
+  l.ws_lse = l.ws_o + up(2 * piece_rows * kD * 4);
+  l.whole_o = l.ws_lse + up(2 * piece_rows * 4);
   l.whole_lse = l.whole_o + up(2 * rows * kD * 4);
   l.prefix = l.whole_lse + up(2 * rows * 4);
-  l.total = l.prefix + up(((size_t)5 * batch + 1) * 4);
+  l.total = l.prefix + up(((size_t)9 * batch + 1) * 4);
   return l;
 }
 
@@ -755,8 +794,9 @@ PKV_API int paged_attention_decode_shared_prefix(
     return fail(PKV_ERR_INVALID_ARG, "%s: num_q_heads %d not a multiple of num_kv_heads %d", fn,
                 num_q_heads, cache.num_kv_heads);
   const int g = num_q_heads / cache.num_kv_heads;
-  if (g > kRows)
-    return fail(PKV_ERR_UNSUPPORTED, "%s: %d query heads per KV head (at most %d)", fn, g, kRows);
+  if (g > kLargeRows)
+    return fail(PKV_ERR_UNSUPPORTED, "%s: %d query heads per KV head (at most %d)", fn, g,
+                kLargeRows);
   if (!(scale == scale)) return fail(PKV_ERR_INVALID_ARG, "%s: scale is NaN", fn);
   if (batch == 0) return PKV_OK;
   if (num_groups <= 0 || num_groups > batch || max_group_size <= 0)
@@ -779,16 +819,6 @@ PKV_API int paged_attention_decode_shared_prefix(
                 workspace_bytes);
 
   const int sms = device_sm_count();
-  const size_t smem = (size_t)kWarps * kWarpSmem + kWarps * kStages * 8 + 1024;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(grouped_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-      return check_launch("paged_attention_decode_shared_prefix: smem attribute");
-    attr_set[dev] = true;
-  }
   const int box_rows = cache.block_size >= kTile ? kTile : cache.block_size;
   const int64_t pool_rows = (int64_t)cache.num_blocks * cache.num_kv_heads * cache.block_size;
   alignas(64) CUtensorMap kmap, vmap;
@@ -807,7 +837,9 @@ PKV_API int paged_attention_decode_shared_prefix(
   p.batch = batch;
   p.num_groups = num_groups;
   p.max_members = max_group_size;
-  p.row_blocks = (max_group_size * g + kRows - 1) / kRows;
+  const bool small = g <= kSmallRows;
+  p.seg_rows = small ? kSmallRows : kLargeRows;
+  p.row_blocks = (max_group_size * g + p.seg_rows - 1) / p.seg_rows;
   p.items = num_groups * p.row_blocks + batch;
   p.num_kv_heads = cache.num_kv_heads;
   p.group = g;
@@ -822,12 +854,12 @@ PKV_API int paged_attention_decode_shared_prefix(
   p.whole_o = reinterpret_cast<float*>(ws + l.whole_o);
   p.whole_lse = reinterpret_cast<float*>(ws + l.whole_lse);
   p.ws_prefix = reinterpret_cast<int32_t*>(ws + l.prefix);
-  p.workers = sms * kWarps;
   p.dbg = dbg_err;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  grouped_decode_kernel<<<sms, kWarps * 32, smem, s>>>(kmap, vmap, p);
-  if (int st = check_launch(fn)) return st;
+  const int st = small ? launch_grouped<kSmallRows / 8, kSmallWarps>(p, kmap, vmap, sms, s)
+                       : launch_grouped<kLargeRows / 8, kLargeWarps>(p, kmap, vmap, sms, s);
+  if (st) return st;
   const int64_t rows = (int64_t)batch * num_q_heads;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((rows + 3) / 4));

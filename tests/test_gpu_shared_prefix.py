@@ -139,6 +139,16 @@ def test_group_query_heads_1_and_8(cuda_device):
         check(case, cuda_device, max_group_size=4)
 
 
+@pytest.mark.parametrize("hq,hkv", [(16, 1), (24, 1), (32, 1), (32, 2)])
+def test_group_query_heads_16_to_32(cuda_device, hq, hkv):
+    # up to 16 query heads per KV head take 16-row segments, more take 32-row ones;
+    # 24 heads make segments that straddle two members
+    case = ragged(f"g{hq // hkv}", 12 + hq, group_sizes=[3, 1, 2], prefix_lens=[300, 17, 64],
+                  suffix_lens=[0, 9, 40, 1, 16, 33], num_q_heads=hq, num_kv_heads=hkv,
+                  peaky=True)
+    check(case, cuda_device)
+
+
 def test_sliding_window_rejected(cuda_device):
     case = ragged("sliding", 10, group_sizes=[2], prefix_lens=[32], suffix_lens=[1, 1])
     case.mask_kind = I.MASK_SLIDING
