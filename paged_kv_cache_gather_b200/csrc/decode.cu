@@ -654,30 +654,34 @@ __global__ void __launch_bounds__(WPC * 32, 1)
 }
 
 // Merges the partials of segments split between workers, and writes zeros /
-// -inf for empty sequences. One warp per (segment, query head): lanes load
-// the pieces' LSEs in parallel, reduce max and sum with shuffles, then sum
-// the weighted partial outputs with lanes over head_dim.
+// -inf for empty sequences. One CTA of kCombineWarps warps per (segment, query
+// head): warp w takes pieces w, w + kCombineWarps, ... of the segment, eight
+// pieces' LSEs and partial outputs in flight at a time, and keeps a running
+// maximum, sum and weighted output (lanes over head_dim); the warps' results
+// are then merged through shared memory, one thread per output element.
+constexpr int kCombineWarps = 4;
 template <int D>
-__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(const DecodeParams p) {
   constexpr int V = D / 32;  // floats per lane
+  constexpr int kBatch = 8;  // pieces in flight per warp
+  static_assert(D <= kCombineWarps * 32, "one thread per output element");
+  __shared__ float sm_m[kCombineWarps], sm_s[kCombineWarps];
+  __shared__ float sm_acc[kCombineWarps][D];
   // launched as a programmatic dependent of the main kernel: wait until its
   // grid has completed and its partials, prefix and outputs are visible
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int lane = threadIdx.x & 31;
-  const int64_t item = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t item = blockIdx.x;
   const int H = p.num_kv_heads;
-  if (item >= (int64_t)p.batch * H * p.group) return;
   const int h = (int)(item % p.group);
   const int64_t seg = item / p.group;
   const int b = (int)(seg / H);
   const int kvh = (int)(seg % H);
   const int n = p.ws_prefix[b + 1] - p.ws_prefix[b];
   const int64_t orow = ((int64_t)b * p.num_q_heads + kvh * p.group + h);
-  __nv_bfloat16* dst = p.out + orow * D + lane * V;
   if (n == 0) {
-#pragma unroll
-    for (int i = 0; i < V; ++i) dst[i] = __float2bfloat16_rn(0.f);
-    if (p.lse && lane == 0) p.lse[orow] = -INFINITY;
+    if (threadIdx.x < D) p.out[orow * D + threadIdx.x] = __float2bfloat16_rn(0.f);
+    if (p.lse && threadIdx.x == 0) p.lse[orow] = -INFINITY;
     return;
   }
   const int64_t T = (int64_t)p.ws_prefix[p.batch] * H;
@@ -693,72 +697,68 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     if (st == en) return -1;
     return (int64_t)w * 2 + ((w == wf && st < s0) ? 1 : 0);
   };
-  // pass 1: log-sum-exp over the pieces, 32 pieces per round
-  float m = -INFINITY, sum = 0.f;
-  for (int base = wf; base <= wl; base += 32) {
-    const int w = base + lane;
-    float x = -INFINITY;
-    if (w <= wl) {
-      const int64_t sl = slot_of(w);
-      if (sl >= 0) x = __ldcg(p.ws_lse + sl * p.group + h);
-    }
-    float mx = x;
-#pragma unroll
-    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const float nm = fmaxf(m, mx);
-    float e = (x == -INFINITY) ? 0.f : __expf(x - nm);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-    sum = (m == -INFINITY ? 0.f : sum * __expf(m - nm)) + e;
-    m = nm;
-  }
-  const float lse = m + logf(sum);
-  // pass 2: weighted sum of the normalised partial outputs
-  float acc[V];
+  float m = -INFINITY, sum = 0.f, acc[V];
 #pragma unroll
   for (int i = 0; i < V; ++i) acc[i] = 0.f;
-  for (int base = wf; base <= wl; base += 32) {
-    const int w = base + lane;
-    int64_t sl = -1;
-    float wgt = 0.f;
-    if (w <= wl) {
-      sl = slot_of(w);
-      if (sl >= 0) wgt = __expf(__ldcg(p.ws_lse + sl * p.group + h) - lse);
-    }
-    // eight pieces' loads in flight at a time (the loop is latency-bound)
-    const int cnt = min(32, wl - base + 1);
-    for (int j0 = 0; j0 < cnt; j0 += 8) {
-      float v[8][V];
-      float wv[8];
+  for (int w0 = wf + warp; w0 <= wl; w0 += kCombineWarps * kBatch) {
+    float x[kBatch], v[kBatch][V];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int j = j0 + u;
-        const float wj = __shfl_sync(0xffffffffu, wgt, j & 31);
-        const int64_t sj = __shfl_sync(0xffffffffu, sl, j & 31);
-        const bool use = j < cnt && sj >= 0;
-        wv[u] = use ? wj : 0.f;
-        const float* src = p.ws_o + ((use ? sj : 0) * p.group + h) * D + lane * V;
-        if constexpr (V == 4) {
-          const float4 x = use ? __ldcg(reinterpret_cast<const float4*>(src))
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-          v[u][0] = x.x;
-          v[u][1] = x.y;
-          v[u][2] = x.z;
-          v[u][3] = x.w;
-        } else {
+    for (int u = 0; u < kBatch; ++u) {
+      const int w = w0 + u * kCombineWarps;
+      const int64_t sl = w <= wl ? slot_of(w) : -1;
+      x[u] = sl >= 0 ? __ldcg(p.ws_lse + sl * p.group + h) : -INFINITY;
+      const float* src = p.ws_o + ((sl >= 0 ? sl : 0) * p.group + h) * D + lane * V;
+      if constexpr (V == 4) {
+        const float4 y = sl >= 0 ? __ldcg(reinterpret_cast<const float4*>(src))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[u][0] = y.x;
+        v[u][1] = y.y;
+        v[u][2] = y.z;
+        v[u][3] = y.w;
+      } else {
 #pragma unroll
-          for (int i = 0; i < V; ++i) v[u][i] = use ? __ldcg(src + i) : 0.f;
-        }
+        for (int i = 0; i < V; ++i) v[u][i] = sl >= 0 ? __ldcg(src + i) : 0.f;
       }
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-#pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] += wv[u] * v[u][i];
     }
+    float nm = m;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) nm = fmaxf(nm, x[u]);
+    if (nm == -INFINITY) continue;
+    const float c = m == -INFINITY ? 0.f : __expf(m - nm);
+    sum *= c;
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[i] *= c;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const float e = x[u] == -INFINITY ? 0.f : __expf(x[u] - nm);
+      sum += e;
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[i] += e * v[u][i];
+    }
+    m = nm;
+  }
+  if (lane == 0) {
+    sm_m[warp] = m;
+    sm_s[warp] = sum;
   }
 #pragma unroll
-  for (int i = 0; i < V; ++i) dst[i] = __float2bfloat16_rn(acc[i]);
-  if (p.lse && lane == 0) p.lse[orow] = lse;
+  for (int i = 0; i < V; ++i) sm_acc[warp][lane * V + i] = acc[i];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) M = fmaxf(M, sm_m[w]);
+    float S = 0.f, A = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) {
+      if (sm_m[w] == -INFINITY) continue;
+      const float c = __expf(sm_m[w] - M);
+      S += sm_s[w] * c;
+      A += sm_acc[w][threadIdx.x] * c;
+    }
+    p.out[orow * D + threadIdx.x] = __float2bfloat16_rn(S > 0.f ? A / S : 0.f);
+    if (p.lse && threadIdx.x == 0) p.lse[orow] = S > 0.f ? M + logf(S) : -INFINITY;
+  }
 }
 
 // ---------------------------------------------------------------- fp32 path
@@ -922,8 +922,8 @@ int launch_bf16_impl(const DecodeArgs& a) {
   if (int st = check_launch("paged_attention_decode")) return st;
   const int64_t items = (int64_t)a.batch * a.cache.num_kv_heads * g;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((items + 3) / 4));
-  cfg.blockDim = dim3(128);
+  cfg.gridDim = dim3((unsigned)items);
+  cfg.blockDim = dim3(kCombineWarps * 32);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = a.stream;
   cudaLaunchAttribute attr[1];
