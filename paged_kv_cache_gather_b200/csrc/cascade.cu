@@ -47,7 +47,6 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kTile = 16;            // tokens per tile
-constexpr int kMaxRows = 32;         // query rows per segment at most (4 n-tiles of 8)
 // Rows per segment and warps per CTA (one CTA per SM). The kernel is
 // latency-bound: 16-row segments (168 registers) let 10 warps fit where 32-row
 // segments (252 registers) allowed 8, 94 us per call on the beams workload
@@ -55,7 +54,6 @@ constexpr int kMaxRows = 32;         // query rows per segment at most (4 n-tile
 // head need 32-row segments.
 constexpr int kSmallRows = 16, kSmallWarps = 10;
 constexpr int kLargeRows = 32, kLargeWarps = 8;
-constexpr int kMaxWarps = kSmallWarps;
 constexpr int kStages = 2;           // TMA ring depth per warp
 constexpr int kMinTilesPerWorker = 2;
 constexpr int kTileBytes = kTile * kD * 2;            // K (or V) bytes of one tile
