@@ -183,23 +183,28 @@ __device__ __forceinline__ void cursor_advance(const DecodeParams& p, Cursor& c)
 // rows x D, 128-byte-swizzled halves of 64 columns). E4M3 pools (KV8, D = 128):
 // a stage is a K tile then a V tile of 16 rows x 128 one-byte codes (one
 // swizzled 128-byte row per token), plus 128 bytes of row scales (K then V)
-// per stage, and each warp owns a f16 work tile that its V tile is decoded
-// into (same layout as a bf16 tile).
+// per stage.
 template <int D, bool KV8 = false>
 struct Cfg {
   static constexpr int kHalves = KV8 ? 1 : D / 64;            // TMA boxes per row
   static constexpr int kTileBytes = kTile * D * (KV8 ? 1 : 2);  // K (or V) bytes of one tile
   static constexpr int kStageBytes = 2 * kTileBytes;           // K then V
-  static constexpr int kWorkBytes = KV8 ? kTile * D * 2 : 0;
   static constexpr int kScaleBytes = KV8 ? 2 * kTile * 4 : 0;
 };
 
 // PH: per-head sliding windows (each head column masks keys below its own
 // start); the instance without them carries none of that code.
 // KV8: E4M3 pools with a float32 scale per stored row (D = 128). Codes are
-// decoded to f16 exactly (cvt.rn.f16x2.e4m3x2) and the MMAs run in f16: K's
-// row scales multiply the scores, V's row scales (times 256, which keeps the
-// products clear of f16 subnormals and is divided out at the end) multiply P.
+// decoded exactly to f16 (cvt.rn.f16x2.e4m3x2) in registers and the MMAs run
+// in f16. K: each ldmatrix word holds four codes of one token, decoded into
+// the A fragments of two k16 steps whose k order the query fragments follow.
+// V: the codes are read transposed (ldmatrix .trans on byte pairs), each word
+// regrouped per head_dim column with a byte permute, so one word gives the
+// A-fragment pairs of two head_dim columns (2r and 2r + 1 of the 16-column
+// block: an accumulator row r holds the column 2r, row r + 8 the column
+// 2r + 1). K's row scales multiply the scores, V's row scales (times 256,
+// which keeps the products clear of f16 subnormals and is divided out at the
+// end) multiply P.
 // APPEND: the decode step's append is fused in. The worker that holds the last
 // tile of a (sequence, KV head) segment writes that sequence's new token
 // (k_new/v_new) into the pools at position seq_lens[b]-1 of its block table
@@ -220,11 +225,10 @@ __global__ void __launch_bounds__(WPC * 32, 1)
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   uint8_t* ring = smem + warp * NSTAGE * C::kStageBytes;
-  uint8_t* work = smem + WPC * NSTAGE * C::kStageBytes + warp * C::kWorkBytes;
-  float* scl = reinterpret_cast<float*>(smem + WPC * (NSTAGE * C::kStageBytes + C::kWorkBytes)) +
+  float* scl = reinterpret_cast<float*>(smem + WPC * NSTAGE * C::kStageBytes) +
                warp * NSTAGE * (C::kScaleBytes / 4);
   uint64_t* bars = reinterpret_cast<uint64_t*>(
-                       smem + WPC * (NSTAGE * (C::kStageBytes + C::kScaleBytes) + C::kWorkBytes)) +
+                       smem + WPC * NSTAGE * (C::kStageBytes + C::kScaleBytes)) +
                    warp * NSTAGE;
 
   const int gw = blockIdx.x * WPC + warp;
@@ -332,6 +336,8 @@ __global__ void __launch_bounds__(WPC * 32, 1)
   const int kco = mi >> 1;                 // +0/+1 chunk for k 0-7 / 8-15
   const int vtok = mr + ((mi >> 1) << 3);  // V tile row (token) this lane addresses
   const int vco = mi & 1;
+  // head_dim columns of accumulator rows g4 and g4 + 8 within a 16-column block
+  const int dlo = KV8 ? 2 * g4 : g4, dhi = KV8 ? 2 * g4 + 1 : g4 + 8;
 
   uint32_t qf[D / 16][2];
   float o[D / 16][4];
@@ -357,21 +363,28 @@ __global__ void __launch_bounds__(WPC * 32, 1)
       // query fragments of this (b, kv head): B operand, column = head g4
       const int hq = cur.kvh * p.group + g4;
       const __nv_bfloat16* qrow = p.q + ((int64_t)cur.b * p.num_q_heads + hq) * D;
+      if constexpr (KV8) {
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        if (g4 < p.group) {
-          if constexpr (KV8) {
+        for (int kk = 0; kk < D / 16; ++kk) {
+          if (g4 < p.group) {
             // f16 B fragments in the k order of the E4M3 A fragments: step kk
             // covers columns 16kk..16kk+15, this lane's four at 16kk + 4*c4
             const uint2 w = __ldg(reinterpret_cast<const uint2*>(qrow + kk * 16 + 4 * c4));
             qf[kk][0] = pack_f16x2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u));
             qf[kk][1] = pack_f16x2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
           } else {
+            qf[kk][0] = qf[kk][1] = 0u;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          if (g4 < p.group) {
             qf[kk][0] = __ldg(reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * c4));
             qf[kk][1] = __ldg(reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8 + 2 * c4));
+          } else {
+            qf[kk][0] = qf[kk][1] = 0u;
           }
-        } else {
-          qf[kk][0] = qf[kk][1] = 0u;
         }
       }
       if (per_head) {
@@ -390,7 +403,7 @@ __global__ void __launch_bounds__(WPC * 32, 1)
     const uint32_t parity = (uint32_t)((k / NSTAGE) & 1);
     uint8_t* kst = ring + stage * C::kStageBytes;
     const uint32_t kbase = smem_u32(kst);
-    const uint32_t vbase = KV8 ? smem_u32(work) : kbase + C::kTileBytes;
+    const uint32_t vbase = kbase + C::kTileBytes;
     if (!mbar_wait(smem_u32(bars + stage), parity)) {
       flag_error(p.dbg, PKV_DBG_TIMEOUT);
       return;
@@ -424,35 +437,7 @@ __global__ void __launch_bounds__(WPC * 32, 1)
         __syncwarp();
       }
     }
-    if constexpr (KV8) {
-      // decode the V codes into the f16 work tile (row r, 16-code chunks
-      // (lane & 1) * 4 ..); rows outside [lo, hi) become zero
-      const int r = lane >> 1;
-      const int pos = tok0 + r;
-      const bool live = pos >= cur.s.lo && pos < cur.s.hi;
-      const uint8_t* vrow = kst + C::kTileBytes + r * 128;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c8 = (lane & 1) * 4 + j;
-        const uint4 w = live ? *reinterpret_cast<const uint4*>(vrow + ((c8 ^ (r & 7)) << 4))
-                             : make_uint4(0u, 0u, 0u, 0u);
-        uint4 lo, hi;
-        lo.x = e4m3x2_to_f16x2(w.x);
-        lo.y = e4m3x2_to_f16x2(w.x >> 16);
-        lo.z = e4m3x2_to_f16x2(w.y);
-        lo.w = e4m3x2_to_f16x2(w.y >> 16);
-        hi.x = e4m3x2_to_f16x2(w.z);
-        hi.y = e4m3x2_to_f16x2(w.z >> 16);
-        hi.z = e4m3x2_to_f16x2(w.w);
-        hi.w = e4m3x2_to_f16x2(w.w >> 16);
-        const int c0 = 2 * c8, c1 = c0 + 1;  // f16 chunks of 8 values
-        *reinterpret_cast<uint4*>(work + (c0 >> 3) * (kTile * 128) + r * 128 +
-                                  (((c0 & 7) ^ (r & 7)) << 4)) = lo;
-        *reinterpret_cast<uint4*>(work + (c1 >> 3) * (kTile * 128) + r * 128 +
-                                  (((c1 & 7) ^ (r & 7)) << 4)) = hi;
-      }
-      __syncwarp();
-    } else if (partial) {
+    if (partial) {
       // rows outside [lo, hi) may hold stale or non-finite data: zero them in V
       for (int i = lane; i < kTile * C::kHalves * 8; i += 32) {
         const int h = i / (kTile * 8);
@@ -577,17 +562,37 @@ __global__ void __launch_bounds__(WPC * 32, 1)
       pb1 = movmatrix_trans(pack_bf16x2(p10, p11));
     }
     // O^T (D x 8) += V^T (D x 16 tokens) * P^T (16 x 8)
+    if constexpr (KV8) {
+      // one transposed load covers two 16-code column blocks: r[0] / r[1] the
+      // first block's tokens 0-7 / 8-15, r[2] / r[3] the second's; each word
+      // holds columns 2g4, 2g4 + 1 of tokens 2c4, 2c4 + 1, regrouped per column
 #pragma unroll
-    for (int mt = 0; mt < D / 16; ++mt) {
-      const int chunk = 2 * mt + vco;
-      const uint32_t addr = vbase + (chunk >> 3) * (kTile * 128) + vtok * 128 +
-                            (((chunk & 7) ^ (vtok & 7)) << 4);
-      uint32_t a[4];
-      ldmatrix_x4_trans(a, addr);
-      if constexpr (KV8)
-        mma_f16_16816(o[mt], a, pb0, pb1);
-      else
+      for (int cp = 0; cp < D / 32; ++cp) {
+        const int chunk = 2 * cp + (mi >> 1);
+        uint32_t r[4];
+        ldmatrix_x4_trans(r, vbase + krow * 128 + ((chunk ^ (krow & 7)) << 4));
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t x0 = byte_perm(r[2 * hh], 0u, 0x3120u);
+          const uint32_t x1 = byte_perm(r[2 * hh + 1], 0u, 0x3120u);
+          uint32_t a[4];
+          a[0] = e4m3x2_to_f16x2(x0);
+          a[1] = e4m3x2_to_f16x2(x0 >> 16);
+          a[2] = e4m3x2_to_f16x2(x1);
+          a[3] = e4m3x2_to_f16x2(x1 >> 16);
+          mma_f16_16816(o[2 * cp + hh], a, pb0, pb1);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        const int chunk = 2 * mt + vco;
+        const uint32_t addr = vbase + (chunk >> 3) * (kTile * 128) + vtok * 128 +
+                              (((chunk & 7) ^ (vtok & 7)) << 4);
+        uint32_t a[4];
+        ldmatrix_x4_trans(a, addr);
         mma_bf16_16816(o[mt], a, pb0, pb1);
+      }
     }
     __syncwarp();
 
@@ -612,14 +617,14 @@ __global__ void __launch_bounds__(WPC * 32, 1)
         const int64_t obase = ((int64_t)cur.b * p.num_q_heads + cur.kvh * p.group) * D;
 #pragma unroll
         for (int mt = 0; mt < D / 16; ++mt) {
-          const int d0 = mt * 16 + g4;
+          const int d0 = mt * 16 + dlo, d1 = mt * 16 + dhi;
           if (h0 < p.group) {
             p.out[obase + h0 * D + d0] = __float2bfloat16_rn(o[mt][0] * inv0);
-            p.out[obase + h0 * D + d0 + 8] = __float2bfloat16_rn(o[mt][2] * inv0);
+            p.out[obase + h0 * D + d1] = __float2bfloat16_rn(o[mt][2] * inv0);
           }
           if (h1 < p.group) {
             p.out[obase + h1 * D + d0] = __float2bfloat16_rn(o[mt][1] * inv1);
-            p.out[obase + h1 * D + d0 + 8] = __float2bfloat16_rn(o[mt][3] * inv1);
+            p.out[obase + h1 * D + d1] = __float2bfloat16_rn(o[mt][3] * inv1);
           }
         }
         if (p.lse && g4 == 0) {
@@ -632,14 +637,14 @@ __global__ void __launch_bounds__(WPC * 32, 1)
         float* wo = p.ws_o + slot * p.group * D;
 #pragma unroll
         for (int mt = 0; mt < D / 16; ++mt) {
-          const int d0 = mt * 16 + g4;
+          const int d0 = mt * 16 + dlo, d1 = mt * 16 + dhi;
           if (h0 < p.group) {
             wo[h0 * D + d0] = o[mt][0] * inv0;
-            wo[h0 * D + d0 + 8] = o[mt][2] * inv0;
+            wo[h0 * D + d1] = o[mt][2] * inv0;
           }
           if (h1 < p.group) {
             wo[h1 * D + d0] = o[mt][1] * inv1;
-            wo[h1 * D + d0 + 8] = o[mt][3] * inv1;
+            wo[h1 * D + d1] = o[mt][3] * inv1;
           }
         }
         if (g4 == 0) {
@@ -866,8 +871,7 @@ int launch_bf16_impl(const DecodeArgs& a) {
   const int workers = sms * WPC;
   const int g = a.num_q_heads / a.cache.num_kv_heads;
   const size_t smem =
-      (size_t)WPC * (NSTAGE * (Cf::kStageBytes + Cf::kScaleBytes) + Cf::kWorkBytes) +
-      WPC * NSTAGE * 8 + 1024;
+      (size_t)WPC * NSTAGE * (Cf::kStageBytes + Cf::kScaleBytes) + WPC * NSTAGE * 8 + 1024;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -938,15 +942,15 @@ int launch_bf16_impl(const DecodeArgs& a) {
 // Warps per CTA (one CTA per SM) and ring depth per warp, the fastest
 // measured on B200: 12 warps with 2-stage rings for bf16 head_dim 128 (192 KB
 // of ring per CTA; 4, 6 and 8 warps with deeper rings were slower), 16 warps
-// with 2-stage rings for E4M3 pools (9% faster than 12 with 3).
+// with 3-stage rings for E4M3 pools (2 stages: within noise; 20 warps spill).
 template <int D>
 int launch_bf16(const DecodeArgs& a) {
   const bool per_head = a.mask.kind == PKV_MASK_SLIDING && a.mask.window_per_head;
   if constexpr (D == 128) {
-    // E4M3 pools: 4 KB tiles and a 4 KB work tile per warp, 197-201 KB per CTA
+    // E4M3 pools: 4 KB stages (+ 128 B of row scales) per warp
     if (a.cache.dtype == PKV_FP8_E4M3) {
       if (per_head) return launch_bf16_impl<D, 3, 12, true, true>(a);
-      return launch_bf16_impl<D, 2, 16, false, true>(a);
+      return launch_bf16_impl<D, 3, 16, false, true>(a);
     }
   }
   if (a.k_new) {

@@ -149,6 +149,13 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Byte permute of {b, a} (a: bytes 0..3, b: bytes 4..7), one selector nibble per result byte.
+__device__ __forceinline__ uint32_t byte_perm(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
 // Two E4M3 codes (bits 0..7 and 8..15 of `x`) to their exact f16 values, the
 // first in bits 0..15 of the result.
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t x) {
