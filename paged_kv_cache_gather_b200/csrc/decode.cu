@@ -659,25 +659,29 @@ __global__ void __launch_bounds__(WPC * 32, 1)
 }
 
 // Merges the partials of segments split between workers, and writes zeros /
-// -inf for empty sequences. One CTA of kCombineWarps warps per (segment, query
-// head): warp w takes pieces w, w + kCombineWarps, ... of the segment, eight
-// pieces' LSEs and partial outputs in flight at a time, and keeps a running
-// maximum, sum and weighted output (lanes over head_dim); the warps' results
-// are then merged through shared memory, one thread per output element.
+// -inf for empty sequences. A CTA has kCombineWarps warps. SPLIT = false: one
+// warp per (segment, query head) item, four items per CTA; SPLIT = true: one
+// CTA per item, warp w taking pieces w, w + kCombineWarps, ... and the warps'
+// results merged through shared memory (for few, long segments, which a
+// single warp would merge over many rounds). Each warp keeps a running
+// maximum, sum and weighted output (lanes over head_dim) with eight pieces'
+// LSEs and partial outputs in flight at a time.
 constexpr int kCombineWarps = 4;
-template <int D>
+template <int D, bool SPLIT>
 __global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(const DecodeParams p) {
   constexpr int V = D / 32;  // floats per lane
   constexpr int kBatch = 8;  // pieces in flight per warp
+  constexpr int kStride = SPLIT ? kCombineWarps : 1;
   static_assert(D <= kCombineWarps * 32, "one thread per output element");
   __shared__ float sm_m[kCombineWarps], sm_s[kCombineWarps];
-  __shared__ float sm_acc[kCombineWarps][D];
+  __shared__ float sm_acc[SPLIT ? kCombineWarps : 1][D];
   // launched as a programmatic dependent of the main kernel: wait until its
   // grid has completed and its partials, prefix and outputs are visible
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t item = blockIdx.x;
+  const int64_t item = SPLIT ? (int64_t)blockIdx.x : (int64_t)blockIdx.x * kCombineWarps + warp;
   const int H = p.num_kv_heads;
+  if (item >= (int64_t)p.batch * H * p.group) return;
   const int h = (int)(item % p.group);
   const int64_t seg = item / p.group;
   const int b = (int)(seg / H);
@@ -685,8 +689,12 @@ __global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(cons
   const int n = p.ws_prefix[b + 1] - p.ws_prefix[b];
   const int64_t orow = ((int64_t)b * p.num_q_heads + kvh * p.group + h);
   if (n == 0) {
-    if (threadIdx.x < D) p.out[orow * D + threadIdx.x] = __float2bfloat16_rn(0.f);
-    if (p.lse && threadIdx.x == 0) p.lse[orow] = -INFINITY;
+    if (SPLIT ? threadIdx.x < D : lane < D / V) {
+      const int t = SPLIT ? threadIdx.x : lane;
+      for (int i = 0; i < (SPLIT ? 1 : V); ++i)
+        p.out[orow * D + (SPLIT ? t : t * V + i)] = __float2bfloat16_rn(0.f);
+    }
+    if (p.lse && (SPLIT ? threadIdx.x == 0 : lane == 0)) p.lse[orow] = -INFINITY;
     return;
   }
   const int64_t T = (int64_t)p.ws_prefix[p.batch] * H;
@@ -705,11 +713,11 @@ __global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(cons
   float m = -INFINITY, sum = 0.f, acc[V];
 #pragma unroll
   for (int i = 0; i < V; ++i) acc[i] = 0.f;
-  for (int w0 = wf + warp; w0 <= wl; w0 += kCombineWarps * kBatch) {
+  for (int w0 = wf + (SPLIT ? warp : 0); w0 <= wl; w0 += kStride * kBatch) {
     float x[kBatch], v[kBatch][V];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      const int w = w0 + u * kCombineWarps;
+      const int w = w0 + u * kStride;
       const int64_t sl = w <= wl ? slot_of(w) : -1;
       x[u] = sl >= 0 ? __ldcg(p.ws_lse + sl * p.group + h) : -INFINITY;
       const float* src = p.ws_o + ((sl >= 0 ? sl : 0) * p.group + h) * D + lane * V;
@@ -742,27 +750,34 @@ __global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(cons
     }
     m = nm;
   }
-  if (lane == 0) {
-    sm_m[warp] = m;
-    sm_s[warp] = sum;
-  }
+  if constexpr (!SPLIT) {
+    const float inv = sum > 0.f ? 1.f / sum : 0.f;
 #pragma unroll
-  for (int i = 0; i < V; ++i) sm_acc[warp][lane * V + i] = acc[i];
-  __syncthreads();
-  if (threadIdx.x < D) {
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kCombineWarps; ++w) M = fmaxf(M, sm_m[w]);
-    float S = 0.f, A = 0.f;
-#pragma unroll
-    for (int w = 0; w < kCombineWarps; ++w) {
-      if (sm_m[w] == -INFINITY) continue;
-      const float c = __expf(sm_m[w] - M);
-      S += sm_s[w] * c;
-      A += sm_acc[w][threadIdx.x] * c;
+    for (int i = 0; i < V; ++i) p.out[orow * D + lane * V + i] = __float2bfloat16_rn(acc[i] * inv);
+    if (p.lse && lane == 0) p.lse[orow] = sum > 0.f ? m + logf(sum) : -INFINITY;
+  } else {
+    if (lane == 0) {
+      sm_m[warp] = m;
+      sm_s[warp] = sum;
     }
-    p.out[orow * D + threadIdx.x] = __float2bfloat16_rn(S > 0.f ? A / S : 0.f);
-    if (p.lse && threadIdx.x == 0) p.lse[orow] = S > 0.f ? M + logf(S) : -INFINITY;
+#pragma unroll
+    for (int i = 0; i < V; ++i) sm_acc[warp][lane * V + i] = acc[i];
+    __syncthreads();
+    if (threadIdx.x < D) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kCombineWarps; ++w) M = fmaxf(M, sm_m[w]);
+      float S = 0.f, A = 0.f;
+#pragma unroll
+      for (int w = 0; w < kCombineWarps; ++w) {
+        if (sm_m[w] == -INFINITY) continue;
+        const float c = __expf(sm_m[w] - M);
+        S += sm_s[w] * c;
+        A += sm_acc[w][threadIdx.x] * c;
+      }
+      p.out[orow * D + threadIdx.x] = __float2bfloat16_rn(S > 0.f ? A / S : 0.f);
+      if (p.lse && threadIdx.x == 0) p.lse[orow] = S > 0.f ? M + logf(S) : -INFINITY;
+    }
   }
 }
 
@@ -925,8 +940,11 @@ int launch_bf16_impl(const DecodeArgs& a) {
                                                                                          p);
   if (int st = check_launch("paged_attention_decode")) return st;
   const int64_t items = (int64_t)a.batch * a.cache.num_kv_heads * g;
+  // segments are split into workers / segments pieces on average: below
+  // eight segments per worker's worth, one warp merges an item in one round
+  const bool split = (int64_t)a.batch * a.cache.num_kv_heads * 8 < workers;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)items);
+  cfg.gridDim = dim3((unsigned)(split ? items : (items + kCombineWarps - 1) / kCombineWarps));
   cfg.blockDim = dim3(kCombineWarps * 32);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = a.stream;
@@ -935,7 +953,10 @@ int launch_bf16_impl(const DecodeArgs& a) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, p);
+  if (split)
+    cudaLaunchKernelEx(&cfg, decode_combine_kernel<D, true>, p);
+  else
+    cudaLaunchKernelEx(&cfg, decode_combine_kernel<D, false>, p);
   return check_launch("paged_attention_decode: combine");
 }
 
