@@ -55,22 +55,23 @@ def peaks():
 # ------------------------------------------------------------------ profiled traffic
 
 # DRAM bytes (read + write) per unit of work, from one ncu capture of each
-# kernel on a smaller case of the same workload (the committed ncu summaries); a full launch
-# scales it by its units. Valid only for the kernel code it was taken on: after
+# kernel (decode: one launch on the full ragged batch; prefill: one launch on
+# one of the four long-context sequences; the committed ncu summaries); a full
+# launch scales it by its units. Valid only for the kernel code it was taken on: after
 # any change to that code (comments aside) the bench reports null until the
 # kernels are profiled again.
 PROFILED_TRAFFIC = {
     "decode": {"sources": ['csrc/decode.cu', 'csrc/pkv_common.cuh'],
-               "code_sha256": "5afabfbef3a6b751c2d3c7b0cf9e1e4d6419c3f09b89f0b53b7df2e6be63dba6",
+               "code_sha256": "4a019026fa74271393fb97970dd63f7ce7d309d5547a4b5eea39b336bc61dda8",
                # per algorithmic byte: one launch of the fused decode step on the full
-               # ragged batch (862712832 B read + 4083712 B written for 860911968 B)
-               "per_unit": (862712832 + 4083712) / 860911968,
+               # ragged batch (862788864 B read + 4375552 B written for 860911968 B)
+               "per_unit": (862788864 + 4375552) / 860911968,
                },
     "prefill": {"sources": ['csrc/prefill.cu', 'csrc/prefill_common.cuh', 'csrc/pkv_common.cuh',
                             'csrc/tc_sm100.cuh'],
-                "code_sha256": "5a03e41c1b52e467e1f8bc793349c8c53fb0b298ac4840a4fddb1e350498b5e5",
+                "code_sha256": "cc231aef4686aba1481fecaf71ca60bc396ce4bf41b59ad77a25f4d4fe2bcc5f",
                 # per causal FLOP: one launch on one long-context sequence
-                "per_unit": (165566976 + 12781568) / 1065168666624,
+                "per_unit": (165521152 + 13004032) / 1065168666624,
                 },
 }
 
