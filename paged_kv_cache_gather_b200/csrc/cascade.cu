@@ -595,59 +595,48 @@ __device__ __forceinline__ float segment_result(const GroupedParams& p, int lane
     if (st == en) return -1;
     return (int64_t)w * 2 + ((w == wf && st < s0) ? 1 : 0);
   };
+  // running maximum, sum and weighted output over the pieces, eight pieces'
+  // LSEs and partial outputs in flight per round (the loop is latency-bound)
   float m = -INFINITY, sum = 0.f;
-  for (int base = wf; base <= wl; base += 32) {
-    const int w = base + lane;
-    float x = -INFINITY;
-    if (w <= wl) {
-      const int64_t sl = slot_of(w);
-      if (sl >= 0) x = __ldcg(p.ws_lse + sl * p.seg_rows + r);
+  for (int w0 = wf; w0 <= wl; w0 += 8) {
+    float x[8];
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int w = w0 + u;
+      const int64_t sl = w <= wl ? slot_of(w) : -1;
+      x[u] = sl >= 0 ? __ldcg(p.ws_lse + sl * p.seg_rows + r) : -INFINITY;
+      v[u] = sl >= 0 ? __ldcg(reinterpret_cast<const float4*>(p.ws_o + (sl * p.seg_rows + r) * kD) +
+                              lane)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    float mx = x;
+    float nm = m;
 #pragma unroll
-    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const float nm = fmaxf(m, mx);
-    float e = (x == -INFINITY) ? 0.f : __expf(x - nm);
+    for (int u = 0; u < 8; ++u) nm = fmaxf(nm, x[u]);
+    if (nm == -INFINITY) continue;
+    const float c = m == -INFINITY ? 0.f : __expf(m - nm);
+    sum *= c;
 #pragma unroll
-    for (int o = 16; o; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-    sum = (m == -INFINITY ? 0.f : sum * __expf(m - nm)) + e;
+    for (int j = 0; j < 4; ++j) acc[j] *= c;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float e = x[u] == -INFINITY ? 0.f : __expf(x[u] - nm);
+      sum += e;
+      acc[0] += e * v[u].x;
+      acc[1] += e * v[u].y;
+      acc[2] += e * v[u].z;
+      acc[3] += e * v[u].w;
+    }
     m = nm;
   }
-  const float lse = m + logf(sum);
-  for (int base = wf; base <= wl; base += 32) {
-    const int w = base + lane;
-    int64_t sl = -1;
-    float wgt = 0.f;
-    if (w <= wl) {
-      sl = slot_of(w);
-      if (sl >= 0) wgt = __expf(__ldcg(p.ws_lse + sl * p.seg_rows + r) - lse);
-    }
-    // eight pieces' loads in flight at a time (the loop is latency-bound)
-    const int cnt = min(32, wl - base + 1);
-    for (int j0 = 0; j0 < cnt; j0 += 8) {
-      float4 v[8];
-      float wv[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int j = j0 + u;
-        const float wj = __shfl_sync(0xffffffffu, wgt, j & 31);
-        const int64_t sj = __shfl_sync(0xffffffffu, sl, j & 31);
-        const bool use = j < cnt && sj >= 0;
-        wv[u] = use ? wj : 0.f;
-        v[u] = use ? __ldcg(reinterpret_cast<const float4*>(p.ws_o + (sj * p.seg_rows + r) * kD) +
-                            lane)
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        acc[0] += wv[u] * v[u].x;
-        acc[1] += wv[u] * v[u].y;
-        acc[2] += wv[u] * v[u].z;
-        acc[3] += wv[u] * v[u].w;
-      }
-    }
+  if (!(sum > 0.f)) {
+    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+    return -INFINITY;
   }
-  return lse;
+  const float inv = 1.f / sum;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) acc[j] *= inv;
+  return m + logf(sum);
 }
 
 }  // namespace
