@@ -159,3 +159,42 @@ def test_unsupported_group_size_is_rejected(cuda_device):
                               block_size=16, num_blocks=4, dtype=torch.bfloat16, seed=2)
     with pytest.raises(pkv.PagedKVError):
         run_decode(case, cuda_device, do_append=False)
+
+
+def poisoned_dead_rows(case, w=0):
+    """Pool rows in the same blocks as visible keys but outside the visible range
+    (past the last key, and before a sliding window's first key) set to NaN."""
+    bs = case.k_cache.shape[2]
+    tab = case.block_tables.numpy()
+    n = 0
+    for b, L in enumerate(case.seq_lens.tolist()):
+        if L <= 0:
+            continue
+        lo = max(0, L - w) if w > 0 else 0
+        dead = list(range(L, -(-L // bs) * bs)) + list(range((lo // bs) * bs, lo))
+        for pos in dead:
+            blk = int(tab[b, pos // bs])
+            case.k_cache[blk, :, pos % bs] = float("nan")
+            case.v_cache[blk, :, pos % bs] = float("nan")
+            n += 1
+    return n
+
+
+@pytest.mark.parametrize("kind,w", [(I.MASK_CAUSAL, 0), (I.MASK_SLIDING, 100)])
+def test_nan_in_rows_outside_the_visible_range(cuda_device, kind, w):
+    # the tile that holds a sequence's last key (or a window's first) also loads
+    # rows the query must not see; stale or non-finite data there changes nothing
+    lens = [5, 17, 300, 1000]
+    nb = sum(-(-L // 16) for L in lens) + 8
+    case = I.make_decode_case(f"nan_rows_{kind}", lens=lens, num_q_heads=32, num_kv_heads=8,
+                              head_dim=128, block_size=16, num_blocks=nb, dtype=torch.bfloat16,
+                              seed=31, mask_kind=kind, window=w)
+    clean = I.PagedCase(**{**case.__dict__})
+    clean.k_cache, clean.v_cache = case.k_cache.clone(), case.v_cache.clone()
+    assert poisoned_dead_rows(case, w) > 0
+    out, lse, _, _ = run_decode(case, cuda_device)
+    # the reference is the attention over the clean pools (the oracle resolves
+    # whole blocks, where the NaN rows would reach its P*V even at weight 0)
+    kc, vc = oracle_after_append(clean)
+    ref_o, ref_l = oracle_decode(clean, kc, vc)
+    assert_attention_close(out, lse, ref_o, ref_l, case.dtype, case.name)

@@ -219,3 +219,29 @@ def test_plain_calls_reject_e4m3_pools(cuda_device):
         pkv.paged_attention_decode(t["q"], torch.from_numpy(kc).to(cuda_device),
                                    torch.from_numpy(vc).to(cuda_device), t["block_tables"],
                                    t["seq_lens"])
+
+
+@pytest.mark.parametrize("w", [0, 100])
+def test_nan_codes_and_scales_outside_the_visible_range(cuda_device, w):
+    # rows of a visible key's tile that the query must not see hold NaN codes
+    # (0x7f) and NaN scales: the decode zeroes them before the P*V product
+    lens = [5, 17, 300, 1000]
+    case = case_of(14 + w, lens, mask=I.MASK_SLIDING if w else I.MASK_CAUSAL, window=w,
+                   peaky=True)
+    kc, vc, ks, vs = quantised_case(case)
+    ref_o, ref_l = oracle_fp8(case, kc, vc, ks, vs)  # on the clean pools
+    bs = kc.shape[2]
+    tab = case.block_tables.numpy()
+    n = 0
+    for b, L in enumerate(lens):
+        lo = max(0, L - w) if w else 0
+        for pos in list(range(L, -(-L // bs) * bs)) + list(range((lo // bs) * bs, lo)):
+            blk = int(tab[b, pos // bs])
+            kc[blk, :, pos % bs] = 0x7F
+            vc[blk, :, pos % bs] = 0x7F
+            ks[blk, :, pos % bs] = np.nan
+            vs[blk, :, pos % bs] = np.nan
+            n += 1
+    assert n > 0
+    out, lse = run_fp8(case, kc, vc, ks, vs, cuda_device)
+    assert_attention_close(out, lse, ref_o, ref_l, torch.bfloat16, "fp8 nan rows")
