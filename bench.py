@@ -62,10 +62,10 @@ def peaks():
 # kernels are profiled again.
 PROFILED_TRAFFIC = {
     "decode": {"sources": ['csrc/decode.cu', 'csrc/pkv_common.cuh'],
-               "code_sha256": "4a019026fa74271393fb97970dd63f7ce7d309d5547a4b5eea39b336bc61dda8",
+               "code_sha256": "359451da6cfdd4e078767c6a8414b2d2c85eed5e4fb0176a917bda3e068e1b80",
                # per algorithmic byte: one launch of the fused decode step on the full
-               # ragged batch (862788864 B read + 4375552 B written for 860911968 B)
-               "per_unit": (862788864 + 4375552) / 860911968,
+               # ragged batch (862692096 B read + 4321792 B written for 860911968 B)
+               "per_unit": (862692096 + 4321792) / 860911968,
                },
     "prefill": {"sources": ['csrc/prefill.cu', 'csrc/prefill_common.cuh', 'csrc/pkv_common.cuh',
                             'csrc/tc_sm100.cuh'],
