@@ -117,3 +117,14 @@ def test_unsupported_pool_dtype_rejected(cuda_device):
     t = to_dev(case, cuda_device)
     with pytest.raises((ValueError, pkv.PagedKVError)):
         fused(case, t, None)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_short_batch(cuda_device, d):
+    # a short list (one tile per warp, segments cut into single-tile pieces),
+    # empty sequences among them, plain and with per-head windows
+    lens = [1, 17, 100, 160, 0, 33]
+    check(ragged(f"append_short_d{d}", lens, d=d, mask_kind=I.MASK_CAUSAL), cuda_device)
+    case = ragged(f"append_short_ph_d{d}", lens, d=d, peaky=True)
+    wph = torch.tensor([0, 5, 64, 1000] * 8, dtype=torch.int32)
+    check(I.with_mask(case, I.MASK_SLIDING, window_per_head=wph), cuda_device)
